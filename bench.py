@@ -1,0 +1,407 @@
+#!/usr/bin/env python
+"""Benchmark of the fused fp32 Linear + epilogue on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+                    [--precision tf32|3xtf32] [--impl fle|reference] [--all]
+
+A step is one fle_forward call over one batch: the tcgen05 contraction with
+its epilogue (plus the -inf fill of out[M] for the pool kind), inputs already
+resident in HBM.  Rank 0 prints one JSON line per config.  Under torchrun
+(N > 1) every rank runs its own replica of the workload (the path shards by
+rows with no exchange): value = all ranks' flops / the slowest rank's time.
+
+--impl reference times the CPU oracle on the host cores instead (a bounded
+sample of rows of the same workload per step).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused Linear+epilogue TFLOP/s and % of roofline per shape, 1×B200"
+
+# name -> (M, K, N, problem)
+CONFIGS = {
+    "linear128x1024x1024_hardtanh_gelu": (128, 1024, 1024, "scale_hardtanh_gelu"),
+    "linear2048x8192x8192_hardtanh_gelu": (2048, 8192, 8192, "scale_hardtanh_gelu"),
+    "linear1024x8192x8192_pool16_gelu_rowmax": (1024, 8192, 8192, "avgpool_gelu_scale_rowmax"),
+    "linear128x32768x32768_swish": (128, 32768, 32768, "swish_scale"),
+    "sweep_m16_k8192_n8192_hardtanh_gelu": (16, 8192, 8192, "scale_hardtanh_gelu"),
+    "sweep_m64_k8192_n8192_hardtanh_gelu": (64, 8192, 8192, "scale_hardtanh_gelu"),
+    "sweep_m256_k8192_n8192_hardtanh_gelu": (256, 8192, 8192, "scale_hardtanh_gelu"),
+    "sweep_m1024_k8192_n8192_hardtanh_gelu": (1024, 8192, 8192, "scale_hardtanh_gelu"),
+    "sweep_m4096_k8192_n8192_hardtanh_gelu": (4096, 8192, 8192, "scale_hardtanh_gelu"),
+}
+DEFAULT_CONFIG = "linear2048x8192x8192_hardtanh_gelu"
+
+L2_BYTES = 126 * 1024 * 1024
+# Nominal dense tensor throughput ratio TF32 : BF16 on B200 (1.1 : 2.25 PFLOP/s).
+TF32_PER_BF16 = 1.1 / 2.25
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "reduction_epilogue_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def profiled_traffic(workload: str, precision: str):
+    """DRAM bytes per launch from the committed ncu summary of this kernel and
+    workload, or None when absent or taken from a different kernel source."""
+    p = os.path.join(ROOT, "profiles", f"fle_gemm_{workload}_{precision}.md")
+    if not os.path.exists(p):
+        return None
+    fields = {}
+    with open(p) as f:
+        for line in f:
+            if ":" in line and line.strip().startswith(("traffic_bytes_per_launch", "source_hash")):
+                k, v = line.split(":", 1)
+                fields[k.strip("- *`").strip()] = v.strip().strip("`")
+    if fields.get("source_hash") != source_hash():
+        return None
+    try:
+        return int(float(fields["traffic_bytes_per_launch"]))
+    except (KeyError, ValueError):
+        return None
+
+
+def algorithmic(M, K, N, problem):
+    flops = 2.0 * M * N * K
+    out_elems = M if problem == "avgpool_gelu_scale_rowmax" else M * N
+    nbytes = 4.0 * (M * K + N * K + N + out_elems)
+    return flops, nbytes, out_elems
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region (NVML, read-only)
+# ----------------------------------------------------------------------------
+REASON_BITS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+    0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+    0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+}
+
+
+class ClockSampler:
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            try:
+                self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+
+    def _reasons(self):
+        nv = self._nv
+        f = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return f(self._h)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = self._reasons()
+                for bit, name in REASON_BITS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if self._h is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": "nvml unavailable"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples), "source": "nvml, 2 ms poll over the timed region"}
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timing (the baseline and the reference arm)
+# ----------------------------------------------------------------------------
+def time_oracle_rows(xh, Wh, bh, problem, rows):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.forward_rows(xh, Wh, bh, rows=rows, **oracle.PROBLEMS[problem])
+    return time.perf_counter() - t0
+
+
+def oracle_sample_rows(xh, Wh, bh, problem, M, budget_s):
+    """Rows to time so one oracle call takes about budget_s seconds."""
+    t1 = time_oracle_rows(xh, Wh, bh, problem, [0])
+    t4 = time_oracle_rows(xh, Wh, bh, problem, list(range(min(4, M))))
+    per_row = max((t4 - t1) / max(min(4, M) - 1, 1), t4 / min(4, M), 1e-6)
+    return max(1, min(M, int(budget_s / per_row)))
+
+
+def cpu_inputs(M, K, N, seed):
+    from reduction_epilogue_b200 import synth
+    x, W, b = synth.linear_inputs(M, K, N, seed=seed, device="cpu")
+    return x.numpy(), W.numpy(), b.numpy()
+
+
+def run_reference(args, name):
+    """The reference arm: the CPU oracle, each step a bounded row sample."""
+    import oracle
+    M, K, N, problem = CONFIGS[name]
+    flops, _, _ = algorithmic(M, K, N, problem)
+    xh, Wh, bh = cpu_inputs(M, K, N, seed=0)
+    per_step_budget = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    R = oracle_sample_rows(xh, Wh, bh, problem, M, per_step_budget)
+    rows = list(range(R))
+    for _ in range(args.warmup):
+        time_oracle_rows(xh, Wh, bh, problem, rows)
+    ts = [time_oracle_rows(xh, Wh, bh, problem, rows) for _ in range(args.steps)]
+    t = sum(ts) / len(ts)
+    step_flops = flops * R / M
+    v = step_flops / t / 1e12
+    sample = f"{R} of {M} rows (full N={N}, K={K}) per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": name, "M": M, "K": K, "N": N, "epilogue": problem, "parallelism": "host cores"},
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# the CUDA path
+# ----------------------------------------------------------------------------
+def run_fle(args, name, dist_ctx):
+    import torch
+
+    import reduction_epilogue_b200 as fle
+    from reduction_epilogue_b200 import synth
+
+    rank, world, dev = dist_ctx
+    M, K, N, problem = CONFIGS[name]
+    flops, nbytes, out_elems = algorithmic(M, K, N, problem)
+    desc = fle.desc_for(problem, args.precision)
+    x, W, b = synth.linear_inputs(M, K, N, seed=rank, device=dev)
+    out = torch.empty((M,) if problem == "avgpool_gelu_scale_rowmax" else (M, N), device=dev)
+    ws_bytes = fle.workspace_size(M, K, N, desc)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    launches_per_step = 2 if problem == "avgpool_gelu_scale_rowmax" else 1
+
+    input_bytes = 4 * (M * K + N * K + N)
+    flush = input_bytes <= 2 * L2_BYTES
+    scrub = torch.empty(2 * L2_BYTES // 4, device=dev) if flush else None
+
+    def step():
+        fle.forward(x, W, b, out, desc, workspace=ws, workspace_bytes=ws_bytes, stream=stream)
+
+    for _ in range(args.warmup):
+        if flush:
+            scrub.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    if fle.device_status(stream) != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index)
+    with sampler:
+        for i in range(args.steps):
+            if flush:
+                scrub.fill_(1.0)
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+    if fle.device_status(stream) != 0:
+        raise RuntimeError("device status set during the timed steps")
+    t_max = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t_max, op=torch.distributed.ReduceOp.MAX)
+    total_ms = float(t_max.item())
+    ms_per_step = total_ms / args.steps
+    value = flops * world * args.steps / (total_ms * 1e-3) / 1e12
+
+    # end to end through the public call: pinned host inputs in, result out
+    e2e = None
+    if not args.no_e2e:
+        xh = x.cpu().pin_memory()
+        Wh = W.cpu().pin_memory()
+        bh = b.cpu().pin_memory()
+        outh = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+        e2e_steps = max(1, min(args.steps, args.e2e_steps))
+        for _ in range(2):
+            x.copy_(xh, non_blocking=True); W.copy_(Wh, non_blocking=True); b.copy_(bh, non_blocking=True)
+            step()
+            outh.copy_(out, non_blocking=True)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            x.copy_(xh, non_blocking=True); W.copy_(Wh, non_blocking=True); b.copy_(bh, non_blocking=True)
+            step()
+            outh.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            torch.distributed.all_reduce(e_ms, op=torch.distributed.ReduceOp.MAX)
+        e2e = {"value": flops * world * e2e_steps / (float(e_ms.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": input_bytes, "d2h_bytes_per_step": 4 * out_elems, "steps": e2e_steps}
+
+    # roofline of the dominant (only) kernel
+    peaks, peak_src = load_peaks()
+    tf32_peak = peaks["bf16_tflops"] * TF32_PER_BF16
+    avg_launch_s = statistics.mean(step_ms) * 1e-3
+    t_tc = flops / (tf32_peak * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    traffic = profiled_traffic(name, args.precision)
+    if t_tc >= t_hbm:
+        achieved = flops / avg_launch_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tf32_peak, "unit": "TFLOP/s",
+                "frac": achieved / tf32_peak,
+                "peak_source": f"{peak_src} bf16 {peaks['bf16_tflops']} TFLOP/s x 1.1/2.25 (TF32:BF16 nominal)"}
+    else:
+        achieved = nbytes / avg_launch_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "peak_source": f"{peak_src} copy bandwidth"}
+    roof["traffic"] = traffic
+    roof["algorithmic_bytes"] = nbytes
+    roof["algorithmic_flops"] = flops
+    roof["roofline_time_us"] = max(t_tc, t_hbm) * 1e6
+    roof["kernel_us_median"] = statistics.median(step_ms) * 1e3
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        import oracle
+        xh = x.cpu().numpy()
+        Wh = W.cpu().numpy()
+        bh = b.cpu().numpy()
+        R = oracle_sample_rows(xh, Wh, bh, problem, M, args.cpu_budget)
+        t = time_oracle_rows(xh, Wh, bh, problem, list(range(R)))
+        cpu = {"value": flops * R / M / t / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+               "kind": "oracle", "sample": f"rows 0..{R - 1} of {M} (full N={N}, K={K}); {t:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "impl": "fle", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "tf32" if args.precision == "tf32" else "3xtf32",
+            "data": "synthetic",
+            "config": {"workload": name, "M": M, "K": K, "N": N, "epilogue": problem, "precision": args.precision,
+                       "l2": "flushed between steps" if flush else "inputs larger than L2",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "plan": fle.plan_string(M, K, N, desc)},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": sampler.summary(),
+            "gpu_launches": launches_per_step * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    del x, W, b, out, ws, scrub
+    torch.cuda.empty_cache()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(CONFIGS))
+    ap.add_argument("--all", action="store_true", help="one line per config")
+    ap.add_argument("--precision", default="tf32", choices=["tf32", "3xtf32"])
+    ap.add_argument("--impl", default="fle", choices=["fle", "reference"])
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work to time")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    names = sorted(CONFIGS) if args.all else [args.config]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        for n in names:
+            run_reference(args, n)
+        return
+
+    import torch
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    import reduction_epilogue_b200 as fle
+    fle.load()
+    try:
+        for n in names:
+            run_fle(args, n, (rank, world, dev))
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

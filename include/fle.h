@@ -1,0 +1,157 @@
+/*
+ * fle.h -- fused fp32 Linear + epilogue on NVIDIA B200 (sm_100a).
+ *
+ * One call computes  y = x * W^T + b  on the tensor cores and applies one of
+ * the epilogues below to each tile while it is still on chip, so only the
+ * final result reaches device memory.  The operation and its three epilogues
+ * are the ones stated by the three pages this library follows:
+ *
+ *   Linear            nn.Linear on x [M,K] with weight W [N,K] and bias b [N]
+ *                     (page "Kimi-K2.6 l2_p98", problem restatement, step 1;
+ *                      page "Kimi-K2.6 l2_p53", task statement, step 1).
+ *   (a) FLE_EPI_SCALE_HARDTANH_GELU
+ *                     out = GELU(clamp(scale * y, clamp_lo, clamp_hi)), exact
+ *                     erf GELU (page "Kimi-K2.6 l2_p53", task statement
+ *                     steps 2-4; the pages' constants are 0.5 and [-2, 2]).
+ *   (b) FLE_EPI_SWISH_SCALE
+ *                     out = y * sigmoid(y) * scale (page "Kimi-K2.6 l2_p59",
+ *                     problem analysis; the page's constant is 2.0).
+ *   (c) FLE_EPI_AVGPOOL_GELU_SCALE_ROWMAX
+ *                     AvgPool1d(pool_k, stride pool_stride, no padding, floor
+ *                     mode) along each row of y, then GELU, then * scale, then
+ *                     the maximum over the pooled row: out [M]
+ *                     (page "Kimi-K2.6 l2_p98", problem restatement steps 2-5;
+ *                      the page's constants are k = 16 and 2.0).
+ *   FLE_EPI_NONE      out = y (the Linear alone).
+ *
+ * All entry points are plain C: host scalars, and device pointers to fp32
+ * data that the caller owns.  Nothing here allocates device memory; scratch
+ * for split-K comes from the caller (fle_workspace_size / workspace).
+ */
+#ifndef FLE_H
+#define FLE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Epilogue kinds (fle_epilogue_desc.kind). */
+typedef enum {
+    FLE_EPI_SCALE_HARDTANH_GELU = 0,
+    FLE_EPI_SWISH_SCALE = 1,
+    FLE_EPI_AVGPOOL_GELU_SCALE_ROWMAX = 2,
+    FLE_EPI_NONE = 3
+} fle_epilogue_kind;
+
+/* Tensor-core precision of the contraction (fle_epilogue_desc.precision).
+ * FLE_PREC_3XTF32: each fp32 operand is split into a TF32 high part and a
+ *   TF32 low part; three products (hi*hi + hi*lo + lo*hi) are accumulated in
+ *   fp32, which is about as accurate as an fp32 FMA dot product.
+ * FLE_PREC_TF32: one TF32 product per term (10-bit mantissa inputs, fp32
+ *   accumulation); three times less tensor work. */
+typedef enum {
+    FLE_PREC_3XTF32 = 0,
+    FLE_PREC_TF32 = 1
+} fle_precision;
+
+/* Parameters of the epilogue.  Fields that a kind does not use are ignored.
+ *   scale              (a), (b), (c): multiplier
+ *   clamp_lo, clamp_hi (a): Hardtanh bounds, clamp_lo <= clamp_hi
+ *   pool_k, pool_stride(c): window and stride; this build supports
+ *                       pool_stride == pool_k with pool_k in {1,2,4,8,16,32} */
+typedef struct {
+    int32_t kind;
+    int32_t precision;
+    float scale;
+    float clamp_lo;
+    float clamp_hi;
+    int32_t pool_k;
+    int32_t pool_stride;
+} fle_epilogue_desc;
+
+/* Status codes. */
+enum {
+    FLE_OK = 0,
+    FLE_ERR_NULL = 1,        /* a required pointer is NULL                   */
+    FLE_ERR_SHAPE = 2,       /* negative size, size >= 2^31, or (c) N < pool_k */
+    FLE_ERR_ALIGN = 3,       /* x or W not 16-byte aligned, K % 4 != 0, or
+                                out / b not 4-byte aligned                   */
+    FLE_ERR_DESC = 4,        /* unknown kind/precision, non-finite scale or
+                                clamp, clamp_lo > clamp_hi, unsupported pool  */
+    FLE_ERR_WORKSPACE = 5,   /* workspace smaller than fle_workspace_size()  */
+    FLE_ERR_ARCH = 6,        /* current device is not sm_100 (B200)          */
+    FLE_ERR_CUDA = 7,        /* a CUDA runtime/driver call failed            */
+    FLE_ERR_TIMEOUT = 8,     /* a device-side bounded wait expired           */
+    FLE_ERR_UNSUPPORTED = 9  /* valid arguments this build does not handle  */
+};
+
+/*
+ * fle_forward -- out = epilogue(x * W^T + b), stream-ordered.
+ *
+ *   x       device, fp32 [M,K] row-major (K contiguous), 16-byte aligned
+ *   W       device, fp32 [N,K] row-major (nn.Linear weight layout), 16-byte aligned
+ *   b       device, fp32 [N], or NULL for no bias
+ *   M,K,N   sizes, each in [0, 2^31); K % 4 == 0 (row pitch must be a
+ *           multiple of 16 bytes for the tensor-memory-access engine)
+ *   desc    host pointer to the epilogue parameters (read during the call only)
+ *   out     device, fp32 [M,N] row-major for (a), (b) and NONE; fp32 [M] for
+ *           (c).  Must not overlap x, W, b or the workspace.
+ *   workspace, workspace_bytes
+ *           device scratch of at least fle_workspace_size(M,K,N,desc) bytes,
+ *           256-byte aligned (may be NULL/0 when that size is 0).  Its contents
+ *           on entry are ignored; it must not be used by another call that
+ *           runs concurrently on the GPU.
+ *   stream  a cudaStream_t (NULL = the legacy default stream)
+ *
+ * Returns FLE_OK once the work is enqueued (no host synchronisation).
+ * Argument errors are detected on the host before anything is enqueued and
+ * leave out untouched.  A device-side failure (a bounded wait that expired)
+ * is recorded in a device status word; read it with fle_device_status().
+ * Sizes M == 0, or N == 0 for the elementwise kinds, are valid and enqueue
+ * nothing.  K == 0 gives out = epilogue(b) (a Linear with no inputs).
+ */
+int fle_forward(const float* x, const float* W, const float* b,
+                int64_t M, int64_t K, int64_t N,
+                const fle_epilogue_desc* desc, float* out,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of caller workspace fle_forward needs for these arguments (0 when
+ * the chosen schedule needs none).  Returns 0 for invalid arguments too;
+ * fle_forward then reports the argument error. */
+size_t fle_workspace_size(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* desc);
+
+/* Static text for a status code; never NULL. */
+const char* fle_status_string(int status);
+
+/* Synchronises `stream`, then returns and clears the device status word of
+ * the current device: FLE_OK, or FLE_ERR_TIMEOUT if a kernel's bounded wait
+ * expired since the last call.  FLE_ERR_CUDA if the synchronisation fails. */
+int fle_device_status(void* stream);
+
+/* Describes the launch plan fle_forward would use, as one line of text
+ * ("tile=128x256 swap=0 splits=1 grid=148 stages=4 ..."), into buf.
+ * Returns FLE_OK or an argument error; does not launch anything. */
+int fle_plan_string(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* desc,
+                    char* buf, size_t buf_bytes);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int fle_version(void);
+
+/*
+ * Test hook for the bounded-wait machinery: launches one CTA whose thread
+ * waits on a shared-memory barrier that nothing ever arrives on, with a wait
+ * limit of timeout_us microseconds.  The wait gives up, records
+ * FLE_ERR_TIMEOUT in the device status word and the kernel returns normally,
+ * so the context stays usable.  Returns the launch status; read the recorded
+ * status with fle_device_status().
+ */
+int fle_test_bounded_wait(uint32_t timeout_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLE_H */

@@ -1,0 +1,362 @@
+// fle_api.cu -- the C ABI of libfle (declared in include/fle.h): argument
+// checks, launch planning, TMA descriptor encoding and kernel launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "fle.h"
+#include "fle_kernel.cuh"
+
+namespace {
+
+using fle::KParams;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool probed = false;
+    bool ok = false;
+    int sms = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int device_info(DeviceInfo* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FLE_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.probed) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return FLE_ERR_CUDA;
+        d.probed = true;
+        d.ok = (major == 10 && minor == 0);
+        d.sms = sms;
+    }
+    if (!d.ok) return FLE_ERR_ARCH;
+    if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return FLE_ERR_CUDA;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    *out = d;
+    return FLE_OK;
+}
+
+// 2-D fp32 K-major operand [rows, K]: box of 32 fp32 (128 bytes) along K by
+// box_rows rows, 128-byte swizzle, out-of-range elements read as zero.
+int encode_operand(CUtensorMap* map, const float* base, int64_t rows, int64_t K, int box_rows) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * sizeof(float)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(fle::kBK), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides,
+                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FLE_OK : FLE_ERR_CUDA;
+}
+
+bool is_pow2_upto32(int k) { return k == 1 || k == 2 || k == 4 || k == 8 || k == 16 || k == 32; }
+
+int check_desc(const fle_epilogue_desc* d) {
+    if (!d) return FLE_ERR_NULL;
+    if (d->kind < FLE_EPI_SCALE_HARDTANH_GELU || d->kind > FLE_EPI_NONE) return FLE_ERR_DESC;
+    if (d->precision != FLE_PREC_3XTF32 && d->precision != FLE_PREC_TF32) return FLE_ERR_DESC;
+    if (d->kind != FLE_EPI_NONE && !std::isfinite(d->scale)) return FLE_ERR_DESC;
+    if (d->kind == FLE_EPI_SCALE_HARDTANH_GELU) {
+        if (!std::isfinite(d->clamp_lo) || !std::isfinite(d->clamp_hi) || d->clamp_lo > d->clamp_hi)
+            return FLE_ERR_DESC;
+    }
+    if (d->kind == FLE_EPI_AVGPOOL_GELU_SCALE_ROWMAX) {
+        if (!is_pow2_upto32(d->pool_k) || d->pool_stride != d->pool_k) return FLE_ERR_DESC;
+    }
+    return FLE_OK;
+}
+
+int check_shape(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d) {
+    const int64_t lim = (int64_t(1) << 31);
+    if (M < 0 || K < 0 || N < 0 || M >= lim || K >= lim || N >= lim) return FLE_ERR_SHAPE;
+    if (d->kind == FLE_EPI_AVGPOOL_GELU_SCALE_ROWMAX && N < d->pool_k) return FLE_ERR_SHAPE;
+    if (K % 4 != 0) return FLE_ERR_ALIGN;
+    return FLE_OK;
+}
+
+struct Plan {
+    bool swap = false;
+    int bn = 256;
+    int prec = fle::kPrecTF32;
+    int stages = 0;
+    int tiles_a = 0, tiles_b = 0;
+    int num_kb = 0, splits = 1, kb_per_split = 0;
+    int units = 0, grid = 0;
+    size_t ws_bytes = 0;
+};
+
+int stages_for(int bn, int prec) {
+    const int stage = (fle::kBM + bn) * fle::kBK * 4 * (prec == fle::kPrec3xTF32 ? 2 : 1);
+    const int s = fle::kSmemStageBudget / stage;
+    return s > 8 ? 8 : s;
+}
+
+Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int sms) {
+    Plan pl;
+    pl.prec = (d->precision == FLE_PREC_3XTF32) ? fle::kPrec3xTF32 : fle::kPrecTF32;
+    pl.swap = (M <= 128) && d->kind != FLE_EPI_AVGPOOL_GELU_SCALE_ROWMAX;
+    if (pl.swap) {
+        pl.bn = M <= 32 ? 32 : (M <= 64 ? 64 : 128);
+    } else {
+        pl.bn = (pl.prec == fle::kPrec3xTF32) ? 128 : 256;
+    }
+    const int64_t Ma = pl.swap ? N : M;
+    const int64_t Nb = pl.swap ? M : N;
+    pl.tiles_a = static_cast<int>((Ma + fle::kBM - 1) / fle::kBM);
+    pl.tiles_b = static_cast<int>((Nb + pl.bn - 1) / pl.bn);
+    pl.num_kb = static_cast<int>((K + fle::kBK - 1) / fle::kBK);
+    pl.splits = 1;
+    pl.kb_per_split = pl.num_kb;
+    pl.units = pl.tiles_a * pl.tiles_b * pl.splits;
+    pl.grid = pl.units < sms ? pl.units : sms;
+    pl.stages = stages_for(pl.bn, pl.prec);
+    pl.ws_bytes = 0;
+    return pl;
+}
+
+template <int BN, int PREC, bool SWAP>
+cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const KParams& p, int grid,
+                        cudaStream_t st) {
+    using C = fle::Cfg<BN, PREC>;
+    auto kern = fle::fle_gemm_kernel<BN, PREC, SWAP>;
+    static bool attr_set[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    kern<<<grid, fle::kThreads, C::kSmemBytes, st>>>(ta, tb, p);
+    return cudaGetLastError();
+}
+
+cudaError_t dispatch(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const KParams& p,
+                     cudaStream_t st) {
+    const bool tf32 = pl.prec == fle::kPrecTF32;
+    if (!pl.swap) {
+        if (tf32 && pl.bn == 256) return launch_gemm<256, fle::kPrecTF32, false>(ta, tb, p, pl.grid, st);
+        if (!tf32 && pl.bn == 128) return launch_gemm<128, fle::kPrec3xTF32, false>(ta, tb, p, pl.grid, st);
+    } else {
+        switch (pl.bn) {
+            case 32:
+                return tf32 ? launch_gemm<32, fle::kPrecTF32, true>(ta, tb, p, pl.grid, st)
+                            : launch_gemm<32, fle::kPrec3xTF32, true>(ta, tb, p, pl.grid, st);
+            case 64:
+                return tf32 ? launch_gemm<64, fle::kPrecTF32, true>(ta, tb, p, pl.grid, st)
+                            : launch_gemm<64, fle::kPrec3xTF32, true>(ta, tb, p, pl.grid, st);
+            case 128:
+                return tf32 ? launch_gemm<128, fle::kPrecTF32, true>(ta, tb, p, pl.grid, st)
+                            : launch_gemm<128, fle::kPrec3xTF32, true>(ta, tb, p, pl.grid, st);
+            default: break;
+        }
+    }
+    return cudaErrorInvalidConfiguration;
+}
+
+uint64_t timeout_ns() {
+    static uint64_t t = [] {
+        const char* e = std::getenv("FLE_TIMEOUT_MS");
+        long ms = e ? std::atol(e) : 0;
+        return static_cast<uint64_t>(ms > 0 ? ms : 1000) * 1000000ull;
+    }();
+    return t;
+}
+
+bool log_enabled() {
+    static bool on = [] {
+        const char* e = std::getenv("FLE_LOG");
+        return e && e[0] == '1';
+    }();
+    return on;
+}
+
+bool sync_check_enabled() {
+    static bool on = [] {
+        const char* e = std::getenv("FLE_SYNC_CHECK");
+        return e && e[0] == '1';
+    }();
+    return on;
+}
+
+int plan_to_string(const Plan& pl, char* buf, size_t n) {
+    if (!buf || n == 0) return FLE_ERR_NULL;
+    std::snprintf(buf, n,
+                  "tile=128x%d swap=%d prec=%s stages=%d tiles=%dx%d kblocks=%d splits=%d kb_per_split=%d "
+                  "units=%d grid=%d workspace=%zu",
+                  pl.bn, pl.swap ? 1 : 0, pl.prec == fle::kPrecTF32 ? "tf32" : "3xtf32", pl.stages,
+                  pl.tiles_a, pl.tiles_b, pl.num_kb, pl.splits, pl.kb_per_split, pl.units, pl.grid,
+                  pl.ws_bytes);
+    return FLE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fle_version(void) { return 100; }
+
+const char* fle_status_string(int s) {
+    switch (s) {
+        case FLE_OK: return "ok";
+        case FLE_ERR_NULL: return "a required pointer is NULL";
+        case FLE_ERR_SHAPE: return "invalid shape (negative, >= 2^31, or N < pool_k for the pool epilogue)";
+        case FLE_ERR_ALIGN: return "misaligned argument (x/W need 16-byte alignment and K % 4 == 0; out/b 4-byte)";
+        case FLE_ERR_DESC: return "invalid epilogue descriptor";
+        case FLE_ERR_WORKSPACE: return "workspace smaller than fle_workspace_size()";
+        case FLE_ERR_ARCH: return "device is not sm_100 (B200)";
+        case FLE_ERR_CUDA: return "a CUDA call failed";
+        case FLE_ERR_TIMEOUT: return "a device-side bounded wait expired";
+        case FLE_ERR_UNSUPPORTED: return "arguments valid but not supported by this build";
+        default: return "unknown status";
+    }
+}
+
+size_t fle_workspace_size(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d) {
+    if (check_desc(d) != FLE_OK || check_shape(M, K, N, d) != FLE_OK) return 0;
+    if (M == 0 || N == 0 || K == 0) return 0;
+    DeviceInfo di;
+    if (device_info(&di) != FLE_OK) return 0;
+    return make_plan(M, K, N, d, di.sms).ws_bytes;
+}
+
+int fle_plan_string(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, char* buf, size_t n) {
+    int st = check_desc(d);
+    if (st != FLE_OK) return st;
+    st = check_shape(M, K, N, d);
+    if (st != FLE_OK) return st;
+    DeviceInfo di;
+    st = device_info(&di);
+    if (st != FLE_OK) return st;
+    return plan_to_string(make_plan(M, K, N, d, di.sms), buf, n);
+}
+
+int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64_t K, int64_t N,
+                const fle_epilogue_desc* d, float* out, void* workspace, size_t workspace_bytes,
+                void* stream) {
+    // ---- host-side argument checks: nothing is enqueued on failure
+    int st = check_desc(d);
+    if (st != FLE_OK) return st;
+    st = check_shape(M, K, N, d);
+    if (st != FLE_OK) return st;
+    const bool pool = d->kind == FLE_EPI_AVGPOOL_GELU_SCALE_ROWMAX;
+    if (M == 0 || (N == 0 && !pool)) return FLE_OK;
+    if (!out) return FLE_ERR_NULL;
+    if (K > 0 && (!x || !W)) return FLE_ERR_NULL;
+    if (K > 0 && ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(W)) & 15u)) return FLE_ERR_ALIGN;
+    if (reinterpret_cast<uintptr_t>(out) & 3u) return FLE_ERR_ALIGN;
+    if (b && (reinterpret_cast<uintptr_t>(b) & 3u)) return FLE_ERR_ALIGN;
+
+    DeviceInfo di;
+    st = device_info(&di);
+    if (st != FLE_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    KParams p{};
+    p.bias = b;
+    p.out = out;
+    p.M = M;
+    p.N = N;
+    p.kind = d->kind;
+    p.scale = d->scale;
+    p.clamp_lo = d->clamp_lo;
+    p.clamp_hi = d->clamp_hi;
+    p.pool_k = pool ? d->pool_k : 1;
+    p.pool_limit = pool ? (N / d->pool_k) * d->pool_k : N;
+    p.vec_out = ((reinterpret_cast<uintptr_t>(out) & 15u) == 0 && N % 4 == 0) ? 1 : 0;
+    p.vec_bias = (b && (reinterpret_cast<uintptr_t>(b) & 15u) == 0) ? 1 : 0;
+    p.timeout_ns = timeout_ns();
+
+    if (K == 0) {
+        const int64_t n = pool ? M : M * N;
+        const int threads = 256;
+        const int64_t blocks = (n + threads - 1) / threads;
+        fle::fle_bias_only_kernel<<<static_cast<unsigned>(blocks), threads, 0, s>>>(p);
+        return cudaGetLastError() == cudaSuccess ? FLE_OK : FLE_ERR_CUDA;
+    }
+
+    const Plan pl = make_plan(M, K, N, d, di.sms);
+    if (pl.ws_bytes > 0) {
+        if (!workspace || workspace_bytes < pl.ws_bytes) return FLE_ERR_WORKSPACE;
+        if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FLE_ERR_ALIGN;
+    }
+    p.Ma = static_cast<int>(pl.swap ? N : M);
+    p.Nb = static_cast<int>(pl.swap ? M : N);
+    p.tiles_a = pl.tiles_a;
+    p.tiles_b = pl.tiles_b;
+    p.num_kb = pl.num_kb;
+    p.splits = pl.splits;
+    p.kb_per_split = pl.kb_per_split;
+    p.num_units = pl.units;
+
+    CUtensorMap ta, tb;
+    const float* A = pl.swap ? W : x;
+    const float* B = pl.swap ? x : W;
+    st = encode_operand(&ta, A, p.Ma, K, fle::kBM);
+    if (st != FLE_OK) return st;
+    st = encode_operand(&tb, B, p.Nb, K, pl.bn);
+    if (st != FLE_OK) return st;
+
+    if (log_enabled()) {
+        char line[256];
+        plan_to_string(pl, line, sizeof line);
+        std::fprintf(stderr, "[fle] M=%lld K=%lld N=%lld kind=%d %s\n", (long long)M, (long long)K,
+                     (long long)N, d->kind, line);
+    }
+
+    if (pool) {
+        const int threads = 256;
+        fle::fle_fill_kernel<<<static_cast<unsigned>((M + threads - 1) / threads), threads, 0, s>>>(
+            out, M, -INFINITY);
+        if (cudaGetLastError() != cudaSuccess) return FLE_ERR_CUDA;
+    }
+    if (dispatch(pl, ta, tb, p, s) != cudaSuccess) return FLE_ERR_CUDA;
+    if (sync_check_enabled()) return fle_device_status(stream);
+    return FLE_OK;
+}
+
+int fle_device_status(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FLE_ERR_CUDA;
+    unsigned h[4] = {0, 0, 0, 0};
+    if (cudaMemcpyFromSymbol(h, fle::g_status, sizeof h) != cudaSuccess) return FLE_ERR_CUDA;
+    if (h[0] != 0) {
+        const unsigned z[4] = {0, 0, 0, 0};
+        if (cudaMemcpyToSymbol(fle::g_status, z, sizeof z) != cudaSuccess) return FLE_ERR_CUDA;
+        if (log_enabled())
+            std::fprintf(stderr, "[fle] device status %u at site %u block %u (count %u)\n", h[0], h[1], h[2], h[3]);
+        return static_cast<int>(h[0]);
+    }
+    return FLE_OK;
+}
+
+int fle_test_bounded_wait(uint32_t timeout_us, void* stream) {
+    DeviceInfo di;
+    int st = device_info(&di);
+    if (st != FLE_OK) return st;
+    fle::fle_bounded_wait_test_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint64_t>(timeout_us) * 1000ull);
+    return cudaGetLastError() == cudaSuccess ? FLE_OK : FLE_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,477 @@
+// fle_kernel.cuh -- the fused Linear + epilogue kernel for sm_100a.
+//
+// One persistent CTA per SM walks a list of work units.  A unit is one output
+// tile (128 rows of operand A x BN rows of operand B) over one range of
+// k-blocks (the whole K unless split-K is on).  Operand A is x and B is W
+// ("direct"), or, for small M, A is W and B is x ("swapped"), so the large
+// dimension sits on the 128-row side of the MMA; either way both operands are
+// K-major, as nn.Linear stores them.
+//
+// Warp roles (256 threads):
+//   warp 0, lane 0   TMA producer: fills a ring of shared-memory stages.
+//   warp 1           allocates TMEM; lane 0 issues the tcgen05.mma chain.
+//   warps 2-3        3xTF32 only: split each landed stage into TF32 hi/lo parts.
+//   warps 4-7        epilogue: TMEM -> registers -> bias + epilogue -> global.
+// The accumulator is double-buffered in TMEM, so the epilogue of one tile
+// overlaps the main loop of the next.
+#pragma once
+
+#include <cuda.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "fle_ptx.cuh"
+
+namespace fle {
+
+constexpr int kBM = 128;           // MMA M: rows of operand A per tile
+constexpr int kBK = 32;            // fp32 per k-block = one 128-byte swizzled row
+constexpr int kUmmaK = 8;          // K of one tcgen05.mma kind::tf32
+constexpr int kThreads = 256;
+constexpr int kSmemStageBudget = 196608;  // bytes of shared memory for stages
+
+enum : int { kEpiHardtanhGelu = 0, kEpiSwish = 1, kEpiPoolMax = 2, kEpiNone = 3 };
+enum : int { kPrec3xTF32 = 0, kPrecTF32 = 1 };
+
+// Wait-site identifiers recorded with a timeout.
+enum : unsigned {
+    kWhereProdEmpty = 1, kWhereMmaFull = 2, kWhereMmaAccEmpty = 3, kWhereEpiAccFull = 4,
+    kWhereConvFull = 5, kWhereDrain = 6, kWhereProdDrain = 7, kWhereTest = 9
+};
+
+struct KParams {
+    const float* bias;      // [N] or nullptr
+    float* out;             // [M,N] or [M]
+    float* ws;              // split-K partial tiles (nullptr when splits == 1)
+    unsigned* counters;     // split-K per-tile arrival counters
+    int64_t M, N;           // output sizes
+    int Ma, Nb;             // rows of operand A and operand B
+    int tiles_a, tiles_b;   // tiles along A rows and along B rows
+    int num_kb;             // k-blocks along K
+    int splits, kb_per_split;
+    int num_units;
+    int kind;
+    float scale, clamp_lo, clamp_hi;
+    int pool_k;
+    int64_t pool_limit;     // columns covered by complete pool windows
+    int vec_out;            // out 16-byte aligned and N % 4 == 0
+    int vec_bias;           // bias 16-byte aligned
+    uint64_t timeout_ns;
+};
+
+template <int BN, int PREC>
+struct Cfg {
+    static constexpr int kABytes = kBM * kBK * 4;
+    static constexpr int kBBytes = BN * kBK * 4;
+    static constexpr int kLoadBytes = kABytes + kBBytes;            // TMA bytes per stage
+    static constexpr int kStageBytes = kLoadBytes * (PREC == kPrec3xTF32 ? 2 : 1);
+    static constexpr int kStagesRaw = kSmemStageBudget / kStageBytes;
+    static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+    static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
+                                    : (2 * BN <= 256) ? 256 : 512;
+    // barriers: full, conv, empty per stage; accf, acce per buffer; drain
+    static constexpr int kNumBars = 3 * kStages + 4 + 1;
+    static constexpr int kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + kNumBars * 8 + 16;
+    static_assert(kStages >= 2, "need at least two stages");
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128 is a multiple of 16 in [16,256]");
+    static_assert(kABytes % 1024 == 0 && kBBytes % 1024 == 0, "tiles must keep 1024-byte alignment");
+};
+
+// ----------------------------------------------------------------------------
+// Epilogue math
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ float gelu_erf(float t) {
+    return t * 0.5f * (1.0f + erff(t * 0.70710678118654752440f));
+}
+
+template <int KIND>
+__device__ __forceinline__ float epi_apply(float y, const KParams& p) {
+    if constexpr (KIND == kEpiHardtanhGelu) {
+        float t = y * p.scale;
+        t = fminf(fmaxf(t, p.clamp_lo), p.clamp_hi);
+        return gelu_erf(t);
+    } else if constexpr (KIND == kEpiSwish) {
+        return (y / (1.0f + expf(-y))) * p.scale;
+    } else {
+        return y;
+    }
+}
+
+// Order-preserving fp32 max through integer atomics (finite values; the
+// target starts at -inf).  Non-negative floats order like signed ints,
+// negative floats order inversely as unsigned ints.
+__device__ __forceinline__ void atomic_max_f32(float* addr, float v) {
+    v = v + 0.0f;  // -0.0 -> +0.0
+    if (v >= 0.0f)
+        atomicMax(reinterpret_cast<int*>(addr), __float_as_int(v));
+    else
+        atomicMin(reinterpret_cast<unsigned*>(addr), __float_as_uint(v));
+}
+
+__device__ __forceinline__ void load_bias32(const KParams& p, int64_t n0, float (&bv)[32]) {
+    if (p.bias == nullptr) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) bv[j] = 0.0f;
+    } else if (p.vec_bias && n0 + 32 <= p.N) {
+        const float4* b4 = reinterpret_cast<const float4*>(p.bias + n0);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float4 t = __ldg(b4 + j);
+            bv[4 * j] = t.x; bv[4 * j + 1] = t.y; bv[4 * j + 2] = t.z; bv[4 * j + 3] = t.w;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) bv[j] = (n0 + j < p.N) ? __ldg(p.bias + n0 + j) : 0.0f;
+    }
+}
+
+// Direct layout, elementwise kinds: this thread holds row m, columns n0..n0+31.
+template <int KIND>
+__device__ __forceinline__ void epi_store_direct(const KParams& p, int64_t m, int64_t n0, float (&v)[32]) {
+    float bv[32];
+    load_bias32(p, n0, bv);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = epi_apply<KIND>(v[j] + bv[j], p);
+    if (m >= p.M) return;
+    float* dst = p.out + m * p.N + n0;
+    if (p.vec_out && n0 + 32 <= p.N) {
+        float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) d4[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (n0 + j < p.N) dst[j] = v[j];
+    }
+}
+
+// Direct layout, pool kind: folds complete windows of this 32-column chunk
+// into the running row maximum.
+__device__ __forceinline__ void epi_pool_direct(const KParams& p, int64_t n0, float (&v)[32], float& best) {
+    float bv[32];
+    load_bias32(p, n0, bv);
+    const int k = p.pool_k;
+    const float inv_k = 1.0f / static_cast<float>(k);
+    float acc = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        acc += v[j] + bv[j];
+        if (((j + 1) & (k - 1)) == 0) {
+            if (n0 + j + 1 <= p.pool_limit) {
+                float g = p.scale * gelu_erf(acc * inv_k);
+                best = fmaxf(best, g);
+            }
+            acc = 0.0f;
+        }
+    }
+}
+
+// Swapped layout: this thread holds output column n, rows m0..m0+31.
+template <int KIND>
+__device__ __forceinline__ void epi_store_swapped(const KParams& p, int64_t n, int64_t m0, float (&v)[32]) {
+    const float bn = (p.bias != nullptr && n < p.N) ? __ldg(p.bias + n) : 0.0f;
+    const bool n_ok = n < p.N;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const float o = epi_apply<KIND>(v[j] + bn, p);
+        if (n_ok && m0 + j < p.M) p.out[(m0 + j) * p.N + n] = o;
+    }
+}
+
+// ----------------------------------------------------------------------------
+// The kernel
+// ----------------------------------------------------------------------------
+template <int BN, int PREC, bool SWAP>
+__global__ void __launch_bounds__(kThreads, 1)
+fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const KParams p) {
+    using C = Cfg<BN, PREC>;
+    constexpr int S = C::kStages;
+    constexpr uint32_t kIdesc = idesc_tf32(kBM, BN);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    auto bar_full = [&](int s) { return smem_u32(bars + s); };
+    auto bar_conv = [&](int s) { return smem_u32(bars + S + s); };
+    auto bar_empty = [&](int s) { return smem_u32(bars + 2 * S + s); };
+    auto bar_accf = [&](int b) { return smem_u32(bars + 3 * S + b); };
+    auto bar_acce = [&](int b) { return smem_u32(bars + 3 * S + 2 + b); };
+    const uint32_t bar_drain = smem_u32(bars + 3 * S + 4);
+    // stage s: [A hi | B hi | A lo | B lo]
+    auto sA = [&](int s) { return sbase + s * C::kStageBytes; };
+    auto sB = [&](int s) { return sbase + s * C::kStageBytes + C::kABytes; };
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(bar_full(s), 1);
+            mbar_init(bar_conv(s), 2);
+            mbar_init(bar_empty(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_accf(b), 1);
+            mbar_init(bar_acce(b), 4);
+        }
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            long long fills = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+                const int ta = u % p.tiles_a;
+                const int rest = u / p.tiles_a;
+                const int tb = rest % p.tiles_b;
+                const int sp = rest / p.tiles_b;
+                const int kb0 = sp * p.kb_per_split;
+                const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait_bounded(bar_empty(stage), phase ^ 1u, abort_flag, p.timeout_ns,
+                                           kWhereProdEmpty)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(bar_full(stage), C::kLoadBytes);
+                    tma_load_2d(sA(stage), &tmA, bar_full(stage), kb * kBK, ta * kBM);
+                    tma_load_2d(sB(stage), &tmB, bar_full(stage), kb * kBK, tb * BN);
+                    ++fills;
+                    if (++stage == S) { stage = 0; phase ^= 1u; }
+                }
+            }
+            // Every issued copy must have landed before the CTA may exit.
+            for (long long f = (fills > S ? fills - S : 0); f < fills; ++f) {
+                const int s = static_cast<int>(f % S);
+                const uint32_t ph = static_cast<uint32_t>((f / S) & 1);
+                volatile int never = 0;
+                mbar_wait_bounded(bar_full(s), ph, &never, p.timeout_ns, kWhereProdDrain);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int buf = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+                const int rest = u / p.tiles_a;
+                const int sp = rest / p.tiles_b;
+                const int kb0 = sp * p.kb_per_split;
+                const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+                if (!mbar_wait_bounded(bar_acce(buf), acc_phase ^ 1u, abort_flag, p.timeout_ns,
+                                       kWhereMmaAccEmpty)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    const uint32_t wbar = (PREC == kPrec3xTF32) ? bar_conv(stage) : bar_full(stage);
+                    if (!mbar_wait_bounded(wbar, phase, abort_flag, p.timeout_ns, kWhereMmaFull)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint64_t a_hi = smem_desc_sw128(sA(stage));
+                    const uint64_t b_hi = smem_desc_sw128(sB(stage));
+#pragma unroll
+                    for (int k = 0; k < kBK / kUmmaK; ++k) {
+                        // advance 8 fp32 = 32 bytes along K inside the swizzle atom
+                        const uint64_t koff = static_cast<uint64_t>(k * 2);
+                        const uint32_t acc = (kb > kb0 || k > 0) ? 1u : 0u;
+                        if constexpr (PREC == kPrec3xTF32) {
+                            const uint64_t a_lo = smem_desc_sw128(sA(stage) + C::kLoadBytes);
+                            const uint64_t b_lo = smem_desc_sw128(sB(stage) + C::kLoadBytes);
+                            mma_tf32(d_tmem, a_lo + koff, b_hi + koff, kIdesc, acc);
+                            mma_tf32(d_tmem, a_hi + koff, b_lo + koff, kIdesc, 1u);
+                            mma_tf32(d_tmem, a_hi + koff, b_hi + koff, kIdesc, 1u);
+                        } else {
+                            mma_tf32(d_tmem, a_hi + koff, b_hi + koff, kIdesc, acc);
+                        }
+                    }
+                    mma_commit(bar_empty(stage));
+                    if (++stage == S) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                mma_commit(bar_accf(buf));
+                buf ^= 1;
+                if (buf == 0) acc_phase ^= 1u;
+            }
+            // All issued MMAs must be complete before TMEM is released.
+            mma_commit(bar_drain);
+            volatile int never = 0;
+            mbar_wait_bounded(bar_drain, 0, &never, p.timeout_ns, kWhereDrain);
+        }
+        __syncwarp();
+    } else if (warp < 4) {
+        // ------------------------------------------------------------ 3xTF32 split
+        if constexpr (PREC == kPrec3xTF32) {
+            const int ct = threadIdx.x - 64;  // 0..63
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+                const int rest = u / p.tiles_a;
+                const int sp = rest / p.tiles_b;
+                const int kb0 = sp * p.kb_per_split;
+                const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    int got = 0;
+                    if (lane == 0)
+                        got = mbar_wait_bounded(bar_full(stage), phase, abort_flag, p.timeout_ns, kWhereConvFull);
+                    got = __shfl_sync(0xffffffffu, got, 0);
+                    if (!got) { ok = false; break; }
+                    // hi = x with the low 13 mantissa bits cleared (exactly a TF32
+                    // value); lo = x - hi (exact in fp32).  hi overwrites x in
+                    // place, lo goes to the same offset in the lo half.
+                    float4* hi4 = reinterpret_cast<float4*>(smem + stage * C::kStageBytes);
+                    float4* lo4 = reinterpret_cast<float4*>(smem + stage * C::kStageBytes + C::kLoadBytes);
+                    constexpr int kVec = C::kLoadBytes / 16;
+#pragma unroll 4
+                    for (int i = ct; i < kVec; i += 64) {
+                        float4 x = hi4[i];
+                        float4 h;
+                        h.x = __uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u);
+                        h.y = __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u);
+                        h.z = __uint_as_float(__float_as_uint(x.z) & 0xFFFFE000u);
+                        h.w = __uint_as_float(__float_as_uint(x.w) & 0xFFFFE000u);
+                        hi4[i] = h;
+                        lo4[i] = make_float4(x.x - h.x, x.y - h.y, x.z - h.z, x.w - h.w);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar_conv(stage));
+                    if (++stage == S) { stage = 0; phase ^= 1u; }
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp - 4;  // TMEM lane quadrant of this warp
+        int buf = 0;
+        uint32_t acc_phase = 0;
+        for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+            const int ta = u % p.tiles_a;
+            const int rest = u / p.tiles_a;
+            const int tb = rest % p.tiles_b;
+            int got = 0;
+            if (lane == 0)
+                got = mbar_wait_bounded(bar_accf(buf), acc_phase, abort_flag, p.timeout_ns, kWhereEpiAccFull);
+            got = __shfl_sync(0xffffffffu, got, 0);
+            if (!got) break;
+            tc_fence_after_sync();
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * BN);
+            if constexpr (!SWAP) {
+                const int64_t m = static_cast<int64_t>(ta) * kBM + q * 32 + lane;
+                float best = -INFINITY;
+                for (int c = 0; c < BN / 32; ++c) {
+                    const int64_t n0 = static_cast<int64_t>(tb) * BN + c * 32;
+                    if (n0 >= p.N) break;  // warp-uniform
+                    float v[32];
+                    tmem_ld32_wait(t_row + c * 32, v);
+                    switch (p.kind) {
+                        case kEpiHardtanhGelu: epi_store_direct<kEpiHardtanhGelu>(p, m, n0, v); break;
+                        case kEpiSwish: epi_store_direct<kEpiSwish>(p, m, n0, v); break;
+                        case kEpiPoolMax: epi_pool_direct(p, n0, v, best); break;
+                        default: epi_store_direct<kEpiNone>(p, m, n0, v); break;
+                    }
+                }
+                if (p.kind == kEpiPoolMax && m < p.M && best > -INFINITY) atomic_max_f32(p.out + m, best);
+            } else {
+                const int64_t n = static_cast<int64_t>(ta) * kBM + q * 32 + lane;
+                for (int c = 0; c < BN / 32; ++c) {
+                    const int64_t m0 = static_cast<int64_t>(tb) * BN + c * 32;
+                    if (m0 >= p.M) break;  // warp-uniform
+                    float v[32];
+                    tmem_ld32_wait(t_row + c * 32, v);
+                    switch (p.kind) {
+                        case kEpiHardtanhGelu: epi_store_swapped<kEpiHardtanhGelu>(p, n, m0, v); break;
+                        case kEpiSwish: epi_store_swapped<kEpiSwish>(p, n, m0, v); break;
+                        default: epi_store_swapped<kEpiNone>(p, n, m0, v); break;
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_acce(buf));
+            buf ^= 1;
+            if (buf == 0) acc_phase ^= 1u;
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
+// K == 0: out = epilogue(b).  One thread per output element (elementwise
+// kinds) or per row (pool kind).
+__global__ void fle_bias_only_kernel(const KParams p) {
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (p.kind == kEpiPoolMax) {
+        if (i >= p.M) return;
+        float best = -INFINITY;
+        for (int64_t w0 = 0; w0 + p.pool_k <= p.pool_limit; w0 += p.pool_k) {
+            float acc = 0.0f;
+            for (int t = 0; t < p.pool_k; ++t) acc += p.bias ? p.bias[w0 + t] : 0.0f;
+            best = fmaxf(best, p.scale * gelu_erf(acc / static_cast<float>(p.pool_k)));
+        }
+        p.out[i] = best;
+        return;
+    }
+    if (i >= p.M * p.N) return;
+    const float y = p.bias ? p.bias[i % p.N] : 0.0f;
+    float o;
+    switch (p.kind) {
+        case kEpiHardtanhGelu: o = epi_apply<kEpiHardtanhGelu>(y, p); break;
+        case kEpiSwish: o = epi_apply<kEpiSwish>(y, p); break;
+        default: o = y; break;
+    }
+    p.out[i] = o;
+}
+
+__global__ void fle_fill_kernel(float* out, int64_t n, float v) {
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i < n) out[i] = v;
+}
+
+// Test hook: one thread waits on a barrier nothing arrives on.
+__global__ void fle_bounded_wait_test_kernel(uint64_t timeout_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0;
+        fence_barrier_init();
+        mbar_wait_bounded(smem_u32(&bar), 0, &abort_flag, timeout_ns, kWhereTest);
+    }
+}
+
+}  // namespace fle

@@ -1,0 +1,106 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry
+point include/fle.h declares, and rejects bad arguments on the host before
+anything reaches a GPU (these run without one)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import reduction_epilogue_b200 as fle
+from reduction_epilogue_b200 import build as fle_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fle_build.build()
+    return fle.load()
+
+
+def declared_functions():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for fn in sorted(os.listdir(inc)):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(inc, fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^[A-Za-z_][\w\s\*]*?\b(fle_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for want in ["fle_forward", "fle_workspace_size", "fle_status_string", "fle_device_status",
+                 "fle_plan_string", "fle_version", "fle_test_bounded_wait"]:
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code in range(0, 10):
+        s = lib.fle_status_string(code)
+        assert s and len(s) > 1
+    assert lib.fle_status_string(12345) == b"unknown status"
+    assert lib.fle_version() >= 100
+
+
+def _call(lib, M, K, N, desc, x=16, W=16, b=None, out=16):
+    # Fake, aligned, non-null "device" addresses: every case below must be
+    # rejected on the host before any pointer is used.
+    return lib.fle_forward(x, W, b, M, K, N, ctypes.byref(desc) if desc is not None else None,
+                           out, None, 0, None)
+
+
+def test_null_and_descriptor_errors(lib):
+    d = fle.desc_for("scale_hardtanh_gelu")
+    assert _call(lib, 4, 8, 8, None) == 1  # FLE_ERR_NULL
+    bad = fle.desc_for("scale_hardtanh_gelu"); bad.kind = 9
+    assert _call(lib, 4, 8, 8, bad) == 4
+    bad = fle.desc_for("scale_hardtanh_gelu"); bad.precision = 5
+    assert _call(lib, 4, 8, 8, bad) == 4
+    bad = fle.desc_for("scale_hardtanh_gelu"); bad.clamp_lo, bad.clamp_hi = 1.0, -1.0
+    assert _call(lib, 4, 8, 8, bad) == 4
+    bad = fle.desc_for("swish_scale"); bad.scale = float("inf")
+    assert _call(lib, 4, 8, 8, bad) == 4
+    bad = fle.desc_for("avgpool_gelu_scale_rowmax"); bad.pool_k = 3; bad.pool_stride = 3
+    assert _call(lib, 4, 8, 64, bad) == 4
+    bad = fle.desc_for("avgpool_gelu_scale_rowmax"); bad.pool_stride = 8
+    assert _call(lib, 4, 8, 64, bad) == 4
+
+
+def test_shape_and_alignment_errors(lib):
+    d = fle.desc_for("scale_hardtanh_gelu")
+    assert _call(lib, -1, 8, 8, d) == 2       # FLE_ERR_SHAPE
+    assert _call(lib, 4, 8, 2**31, d) == 2
+    assert _call(lib, 4, 6, 8, d) == 3        # K % 4 != 0 -> FLE_ERR_ALIGN
+    p = fle.desc_for("avgpool_gelu_scale_rowmax")
+    assert _call(lib, 4, 8, 15, p) == 2       # N < pool_k
+    assert _call(lib, 4, 8, 8, d, x=17) == 3  # x not 16-byte aligned
+    assert _call(lib, 4, 8, 8, d, W=24) == 3
+    assert _call(lib, 4, 8, 8, d, out=18) == 3
+    assert _call(lib, 4, 8, 8, d, out=None) == 1
+    assert _call(lib, 4, 8, 8, d, x=None) == 1
+
+
+def test_empty_sizes_enqueue_nothing(lib):
+    d = fle.desc_for("scale_hardtanh_gelu")
+    # M == 0, or N == 0 for an elementwise kind, is valid and returns before
+    # touching the device (no device exists here).
+    assert _call(lib, 0, 8, 8, d, x=None, W=None, out=None) == 0
+    assert _call(lib, 4, 8, 0, d, x=None, W=None, out=None) == 0
+    assert lib.fle_workspace_size(0, 8, 8, ctypes.byref(d)) == 0
+    assert lib.fle_workspace_size(4, 6, 8, ctypes.byref(d)) == 0
+
+
+def test_binding_raises_with_status():
+    d = fle.desc_for("scale_hardtanh_gelu")
+    with pytest.raises(fle.FleError) as e:
+        fle.forward(16, 16, None, 16, d, M=-1, K=8, N=8, stream=0)
+    assert e.value.status == 2

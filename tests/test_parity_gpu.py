@@ -1,0 +1,236 @@
+"""GPU parity: the CUDA library, called through its C ABI, against the CPU
+oracle on the same seeded inputs.
+
+Tolerances (elementwise, ref = oracle):
+  3xTF32   |got - ref| <= 1e-4 + 1e-4 |ref|
+  TF32     |got - ref| <= 5e-3 + 5e-3 |ref|
+Small shapes (several tiles plus ragged tails, both the direct and the
+swapped operand order) are compared in full; the full-size workloads on a
+seeded sample of whole rows, in the same launch plan the benchmark times.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from reduction_epilogue_b200 import synth
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+TOL = {"3xtf32": (1e-4, 1e-4), "tf32": (5e-3, 5e-3)}
+
+
+@pytest.fixture(scope="module")
+def fle():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    import reduction_epilogue_b200 as m
+    from reduction_epilogue_b200 import build
+    build.build()
+    m.load()
+    return m
+
+
+def _oracle(x, W, b, problem, rows=None):
+    return oracle.forward_rows(x.cpu().numpy(), W.cpu().numpy(), None if b is None else b.cpu().numpy(),
+                               rows=rows, **oracle.PROBLEMS[problem])
+
+
+def _assert_close(got, ref, precision, what=""):
+    atol, rtol = TOL[precision]
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape
+    assert np.isfinite(got).all(), what + ": non-finite output"
+    err = np.abs(got - ref)
+    bound = atol + rtol * np.abs(ref)
+    bad = err > bound
+    if bad.any():
+        i = np.unravel_index(np.argmax(err - bound), err.shape)
+        pytest.fail(f"{what}: {int(bad.sum())} of {bad.size} outside tolerance; worst at {i}: "
+                    f"got {got[i]!r} ref {ref[i]!r} err {err[i]:.3e} bound {bound[i]:.3e}")
+
+
+def _run(fle, x, W, b, problem, precision):
+    out = fle.linear_epilogue(x, W, b, problem, precision)
+    torch.cuda.synchronize()
+    assert fle.device_status() == 0
+    return out
+
+
+SMALL = [(1, 4, 1), (7, 36, 33), (16, 64, 130), (33, 100, 257), (128, 1024, 1024),
+         (130, 68, 300), (257, 260, 520), (300, 132, 1000)]
+PROBLEMS = ["scale_hardtanh_gelu", "swish_scale", "avgpool_gelu_scale_rowmax", "none"]
+
+
+@pytest.mark.parametrize("precision", ["tf32", "3xtf32"])
+@pytest.mark.parametrize("problem", PROBLEMS)
+@pytest.mark.parametrize("M,K,N", SMALL)
+def test_small_full_compare(fle, M, K, N, problem, precision):
+    if problem == "avgpool_gelu_scale_rowmax" and N < 16:
+        pytest.skip("pool needs N >= 16")
+    x, W, b = synth.linear_inputs(M, K, N, seed=M + 7 * K + 13 * N, device="cuda")
+    out = _run(fle, x, W, b, problem, precision)
+    _assert_close(out.cpu().numpy(), _oracle(x, W, b, problem), precision, f"{problem} {M}x{K}x{N}")
+
+
+# Full-size workloads: (M, K, N, problem, sampled rows)
+FULL = [
+    (2048, 8192, 8192, "scale_hardtanh_gelu", 64),
+    (1024, 8192, 8192, "avgpool_gelu_scale_rowmax", 64),
+    (128, 32768, 32768, "swish_scale", 48),
+    (128, 1024, 1024, "scale_hardtanh_gelu", 128),
+] + [(m, 8192, 8192, "scale_hardtanh_gelu", 24) for m in (16, 64, 256, 1024, 4096)]
+
+
+@pytest.mark.parametrize("precision", ["tf32", "3xtf32"])
+@pytest.mark.parametrize("M,K,N,problem,nrows", FULL)
+def test_full_size_sampled_rows(fle, M, K, N, problem, nrows, precision):
+    x, W, b = synth.linear_inputs(M, K, N, seed=0, device="cuda")
+    out = _run(fle, x, W, b, problem, precision)
+    rows = synth.sample_rows(M, nrows, seed=1)
+    got = out.cpu().numpy()[rows]
+    ref = _oracle(x, W, b, problem, rows=rows)
+    _assert_close(got, ref, precision, f"{problem} {M}x{K}x{N} rows={len(rows)}")
+    del x, W, b, out
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("precision", ["tf32", "3xtf32"])
+@pytest.mark.parametrize("M,K,N", [(300, 1024, 520), (100, 1024, 300), (5, 2048, 77)])
+def test_integer_inputs_are_exact(fle, M, K, N, precision):
+    # Integers in [-4, 4] are exact in TF32; every partial sum stays below 2^24,
+    # so the contraction is exact in any order: bit-exact against the oracle.
+    x, W, b = synth.integer_inputs(M, K, N, seed=4, device="cuda")
+    out = _run(fle, x, W, b, "none", precision)
+    ref = _oracle(x, W, b, "none")
+    np.testing.assert_array_equal(out.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("precision", ["tf32", "3xtf32"])
+@pytest.mark.parametrize("M", [64, 512])
+def test_hardtanh_saturation(fle, M, precision):
+    # x ~ N(0, 50^2) drives most of 0.5*y past +-2: both clamp branches fire.
+    K, N = 256, 384
+    x, W, b = synth.linear_inputs(M, K, N, seed=9, device="cuda", x_std=50.0)
+    out = _run(fle, x, W, b, "scale_hardtanh_gelu", precision)
+    ref = _oracle(x, W, b, "scale_hardtanh_gelu")
+    assert (ref > 1.95).mean() > 0.1 and (ref < -0.045).mean() > 0.1
+    _assert_close(out.cpu().numpy(), ref, precision, "saturation")
+
+
+def test_gelu_is_the_erf_form(fle):
+    # y = W[:, 0] exactly (x = e0, no bias).  Where tanh-GELU and erf-GELU
+    # differ by more than 2e-4 inside the clamp range, the 3xTF32 result must
+    # follow erf-GELU to 1e-4 + 1e-4|ref|.
+    ts = np.linspace(-2.0, 2.0, 4001)
+    tanh_g = 0.5 * ts * (1 + np.tanh(math.sqrt(2 / math.pi) * (ts + 0.044715 * ts ** 3)))
+    erf_g = np.array([oracle.gelu(t) for t in ts])
+    pick = ts[np.abs(tanh_g - erf_g) > 2e-4]
+    assert pick.size > 0
+    N = int(pick.size)
+    W = torch.zeros(N, 4, dtype=torch.float32)
+    W[:, 0] = torch.from_numpy(2.0 * pick).float()  # y = 2t so that 0.5*y = t
+    x = torch.zeros(3, 4, dtype=torch.float32)
+    x[:, 0] = 1.0
+    x, W = x.cuda(), W.cuda()
+    out = _run(fle, x, W, None, "scale_hardtanh_gelu", "3xtf32")
+    ref = _oracle(x, W, None, "scale_hardtanh_gelu")
+    _assert_close(out.cpu().numpy(), ref, "3xtf32", "erf-GELU")
+    tanh_ref = 0.5 * 2 * pick * 0.5 * (1 + np.tanh(math.sqrt(2 / math.pi) * (pick + 0.044715 * pick ** 3)))
+    assert np.abs(out.cpu().numpy()[0] - tanh_ref).max() > 1.5e-4
+
+
+def test_pool_max_after_gelu(fle):
+    # Two windows with means -3 and -0.75: the row max of GELU*2 is
+    # 2*GELU(-3) ~ -0.0081, not 2*GELU(-0.75) ~ -0.34.
+    N, K = 32, 4
+    W = torch.zeros(N, K)
+    W[:16, 0] = -3.0
+    W[16:, 0] = -0.75
+    x = torch.zeros(2, K)
+    x[:, 0] = 1.0
+    out = _run(fle, x.cuda(), W.cuda(), None, "avgpool_gelu_scale_rowmax", "3xtf32")
+    ref = _oracle(x, W, None, "avgpool_gelu_scale_rowmax")
+    _assert_close(out.cpu().numpy(), ref, "3xtf32", "pool order")
+    assert abs(float(out[0]) - 2 * oracle.gelu(-3.0)) < 1e-5
+
+
+@pytest.mark.parametrize("problem", PROBLEMS)
+def test_k_zero_gives_epilogue_of_bias(fle, problem):
+    M, N = 5, 48
+    _, _, b = synth.linear_inputs(M, 4, N, seed=3, device="cuda")
+    b = b * 10
+    x = torch.empty(M, 0, device="cuda")
+    W = torch.empty(N, 0, device="cuda")
+    out = _run(fle, x, W, b, problem, "tf32")
+    ref = _oracle(x, W, b, problem)
+    _assert_close(out.cpu().numpy(), ref, "3xtf32", "K=0")
+
+
+def test_no_bias(fle):
+    x, W, _ = synth.linear_inputs(200, 96, 260, seed=12, device="cuda")
+    out = _run(fle, x, W, None, "swish_scale", "3xtf32")
+    _assert_close(out.cpu().numpy(), _oracle(x, W, None, "swish_scale"), "3xtf32", "no bias")
+
+
+def test_empty_m_is_a_no_op(fle):
+    x = torch.empty(0, 64, device="cuda")
+    W = torch.randn(32, 64, device="cuda")
+    out = fle.linear_epilogue(x, W, None, "scale_hardtanh_gelu")
+    assert out.shape == (0, 32)
+
+
+def test_misaligned_operand_is_rejected(fle):
+    base = torch.zeros(4 * 64 + 1, device="cuda")
+    x = base[1:].view(4, 64)  # 4-byte offset: not 16-byte aligned
+    W = torch.zeros(8, 64, device="cuda")
+    with pytest.raises(fle.FleError) as e:
+        fle.linear_epilogue(x, W, None, "none")
+    assert e.value.status == 3
+
+
+def test_repeat_calls_are_deterministic(fle):
+    x, W, b = synth.linear_inputs(512, 1024, 2048, seed=5, device="cuda")
+    a = _run(fle, x, W, b, "avgpool_gelu_scale_rowmax", "tf32")
+    c = _run(fle, x, W, b, "avgpool_gelu_scale_rowmax", "tf32")
+    assert torch.equal(a, c)
+    a = _run(fle, x, W, b, "scale_hardtanh_gelu", "3xtf32")
+    c = _run(fle, x, W, b, "scale_hardtanh_gelu", "3xtf32")
+    assert torch.equal(a, c)
+
+
+def test_bounded_wait_expires_cleanly(fle):
+    # A barrier nothing arrives on: the wait gives up after 2 ms, records
+    # FLE_ERR_TIMEOUT and the kernel returns; the context stays usable.
+    lib = fle.load()
+    assert lib.fle_test_bounded_wait(2000, None) == 0
+    assert fle.device_status() == 8
+    assert fle.device_status() == 0
+    x, W, b = synth.linear_inputs(64, 64, 64, seed=1, device="cuda")
+    out = _run(fle, x, W, b, "none", "3xtf32")
+    _assert_close(out.cpu().numpy(), _oracle(x, W, b, "none"), "3xtf32", "after timeout")
+
+
+def test_plan_choices(fle):
+    d = fle.desc_for("swish_scale", "tf32")
+    assert "swap=1" in fle.plan_string(128, 32768, 32768, d)
+    d = fle.desc_for("scale_hardtanh_gelu", "tf32")
+    assert "swap=0" in fle.plan_string(2048, 8192, 8192, d)
+
+
+def test_tf32_input_conversion_probe(fle, capsys):
+    # Records how the tensor core reads an fp32 operand in kind::tf32 (the low
+    # 13 mantissa bits dropped, or rounded).  Informational; the 3xTF32 split
+    # masks the high part explicitly, so it depends on neither behaviour.
+    v = 1.0 + 2.0 ** -11 + 2.0 ** -12
+    x = torch.full((1, 4), v, device="cuda")
+    W = torch.ones(1, 4, device="cuda")
+    out = _run(fle, x, W, None, "none", "tf32")
+    got = float(out[0, 0])
+    trunc, rn = 4.0, 4.0 * (1.0 + 2.0 ** -10)
+    assert got in (trunc, rn), got
+    with capsys.disabled():
+        print(f"\n[tf32 operand conversion: {'truncate' if got == trunc else 'round-to-nearest'}]")
