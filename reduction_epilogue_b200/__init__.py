@@ -16,7 +16,7 @@ import os
 __all__ = [
     "EPI_SCALE_HARDTANH_GELU", "EPI_SWISH_SCALE", "EPI_AVGPOOL_GELU_SCALE_ROWMAX", "EPI_NONE",
     "PREC_3XTF32", "PREC_TF32", "EpilogueDesc", "FleError", "desc_for", "forward",
-    "workspace_size", "device_status", "plan_string", "linear_epilogue", "library_path", "load",
+    "workspace_size", "device_status", "plan_string", "plan_units", "linear_epilogue", "library_path", "load",
     "PROBLEMS",
 ]
 
@@ -95,6 +95,9 @@ def load():
     lib.fle_plan_string.restype = ctypes.c_int
     lib.fle_version.argtypes = []
     lib.fle_version.restype = ctypes.c_int
+    lib.fle_plan_units.argtypes = [i64, i64, i64, ctypes.POINTER(EpilogueDesc), ctypes.c_int, ctypes.c_int,
+                                   vp, ctypes.c_int, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
+    lib.fle_plan_units.restype = ctypes.c_int
     lib.fle_test_bounded_wait.argtypes = [ctypes.c_uint32, vp]
     lib.fle_test_bounded_wait.restype = ctypes.c_int
     _lib = lib
@@ -160,6 +163,23 @@ def plan_string(M: int, K: int, N: int, desc: EpilogueDesc) -> str:
     if st != FLE_OK:
         raise FleError(st, "fle_plan_string")
     return buf.value.decode()
+
+
+def plan_units(M: int, K: int, N: int, desc: EpilogueDesc, num_sms: int, cta: int):
+    """(grid, [unit rows]) that CTA `cta` would run; see fle_plan_units."""
+    import numpy as np
+    lib = load()
+    n = ctypes.c_int(0)
+    g = ctypes.c_int(0)
+    st = lib.fle_plan_units(M, K, N, ctypes.byref(desc), num_sms, cta, None, 0, ctypes.byref(n), ctypes.byref(g))
+    if st != FLE_OK:
+        raise FleError(st, "fle_plan_units")
+    rows = np.zeros((max(n.value, 1), 10), dtype=np.int32)
+    st = lib.fle_plan_units(M, K, N, ctypes.byref(desc), num_sms, cta, rows.ctypes.data, n.value,
+                            ctypes.byref(n), ctypes.byref(g))
+    if st != FLE_OK:
+        raise FleError(st, "fle_plan_units")
+    return g.value, rows[: n.value]
 
 
 def device_status(stream=None) -> int:

@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -100,16 +101,31 @@ struct Plan {
     int bn = 256;
     int prec = fle::kPrecTF32;
     int stages = 0;
-    int tiles_a = 0, tiles_b = 0;
-    int num_kb = 0, splits = 1, kb_per_split = 0;
-    int units = 0, grid = 0;
-    size_t ws_bytes = 0;
+    int tiles_a = 0, tiles_b = 0, tiles = 0;
+    int num_kb = 0;
+    int dp_tiles = 0;          // tiles done whole, one CTA each
+    int64_t sk_iters = 0;      // k-blocks of the remaining tiles, spread over the grid
+    int sk_tiles = 0;
+    int grid = 0;
+    size_t partial_bytes = 0;  // workspace: 2 partial tiles per CTA ...
+    size_t ws_bytes = 0;       // ... then one arrival counter per stream-K tile
 };
 
 int stages_for(int bn, int prec) {
     const int stage = (fle::kBM + bn) * fle::kBK * 4 * (prec == fle::kPrec3xTF32 ? 2 : 1);
     const int s = fle::kSmemStageBudget / stage;
     return s > 8 ? 8 : s;
+}
+
+// Fewest k-blocks (of 32) a CTA takes in the stream-K part of a schedule.
+constexpr int64_t kMinSkIters = 16;
+
+const char* sched_override() {
+    static const char* v = [] {
+        const char* e = std::getenv("FLE_SCHED");
+        return e ? e : "";
+    }();
+    return v;
 }
 
 Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int sms) {
@@ -125,13 +141,36 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
     const int64_t Nb = pl.swap ? M : N;
     pl.tiles_a = static_cast<int>((Ma + fle::kBM - 1) / fle::kBM);
     pl.tiles_b = static_cast<int>((Nb + pl.bn - 1) / pl.bn);
+    pl.tiles = pl.tiles_a * pl.tiles_b;
     pl.num_kb = static_cast<int>((K + fle::kBK - 1) / fle::kBK);
-    pl.splits = 1;
-    pl.kb_per_split = pl.num_kb;
-    pl.units = pl.tiles_a * pl.tiles_b * pl.splits;
-    pl.grid = pl.units < sms ? pl.units : sms;
     pl.stages = stages_for(pl.bn, pl.prec);
-    pl.ws_bytes = 0;
+
+    const int64_t T = pl.tiles;
+    const int64_t G = sms;
+    const int64_t iters = T * pl.num_kb;
+    const bool force_dp = std::strcmp(sched_override(), "dp") == 0;
+    pl.dp_tiles = static_cast<int>(T);
+    pl.grid = static_cast<int>(T < G ? T : G);
+    if (!force_dp && T % G != 0 && pl.num_kb >= kMinSkIters) {
+        if (T > G) {
+            // keep all but the last full wave data-parallel; the last full wave
+            // plus the partial one are spread evenly over every CTA
+            pl.dp_tiles = static_cast<int>((T / G - 1) * G);
+            pl.grid = static_cast<int>(G);
+        } else {
+            const int64_t g_sk = std::min<int64_t>(G, iters / kMinSkIters);
+            if (g_sk > T) {
+                pl.dp_tiles = 0;
+                pl.grid = static_cast<int>(g_sk);
+            }
+        }
+    }
+    pl.sk_tiles = static_cast<int>(T - pl.dp_tiles);
+    pl.sk_iters = static_cast<int64_t>(pl.sk_tiles) * pl.num_kb;
+    if (pl.sk_tiles > 0) {
+        pl.partial_bytes = static_cast<size_t>(2) * pl.grid * fle::kBM * pl.bn * sizeof(float);
+        pl.ws_bytes = pl.partial_bytes + ((static_cast<size_t>(pl.sk_tiles) * 4 + 255) & ~size_t(255));
+    }
     return pl;
 }
 
@@ -203,10 +242,10 @@ bool sync_check_enabled() {
 int plan_to_string(const Plan& pl, char* buf, size_t n) {
     if (!buf || n == 0) return FLE_ERR_NULL;
     std::snprintf(buf, n,
-                  "tile=128x%d swap=%d prec=%s stages=%d tiles=%dx%d kblocks=%d splits=%d kb_per_split=%d "
-                  "units=%d grid=%d workspace=%zu",
+                  "tile=128x%d swap=%d prec=%s stages=%d tiles=%dx%d kblocks=%d dp_tiles=%d sk_tiles=%d "
+                  "sk_kblocks=%lld grid=%d workspace=%zu",
                   pl.bn, pl.swap ? 1 : 0, pl.prec == fle::kPrecTF32 ? "tf32" : "3xtf32", pl.stages,
-                  pl.tiles_a, pl.tiles_b, pl.num_kb, pl.splits, pl.kb_per_split, pl.units, pl.grid,
+                  pl.tiles_a, pl.tiles_b, pl.num_kb, pl.dp_tiles, pl.sk_tiles, (long long)pl.sk_iters, pl.grid,
                   pl.ws_bytes);
     return FLE_OK;
 }
@@ -306,9 +345,13 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
     p.tiles_a = pl.tiles_a;
     p.tiles_b = pl.tiles_b;
     p.num_kb = pl.num_kb;
-    p.splits = pl.splits;
-    p.kb_per_split = pl.kb_per_split;
-    p.num_units = pl.units;
+    p.num_tiles = pl.tiles;
+    p.dp_tiles = pl.dp_tiles;
+    p.sk_iters = pl.sk_iters;
+    if (pl.sk_tiles > 0) {
+        p.ws = static_cast<float*>(workspace);
+        p.counters = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + pl.partial_bytes);
+    }
 
     CUtensorMap ta, tb;
     const float* A = pl.swap ? W : x;
@@ -325,14 +368,58 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
                      (long long)N, d->kind, line);
     }
 
-    if (pool) {
+    if (pool || pl.sk_tiles > 0) {
         const int threads = 256;
-        fle::fle_fill_kernel<<<static_cast<unsigned>((M + threads - 1) / threads), threads, 0, s>>>(
-            out, M, -INFINITY);
+        const int64_t n = std::max<int64_t>(pool ? M : 0, pl.sk_tiles);
+        fle::fle_prep_kernel<<<static_cast<unsigned>((n + threads - 1) / threads), threads, 0, s>>>(
+            pool ? out : nullptr, pool ? M : 0, p.counters, pl.sk_tiles);
         if (cudaGetLastError() != cudaSuccess) return FLE_ERR_CUDA;
     }
     if (dispatch(pl, ta, tb, p, s) != cudaSuccess) return FLE_ERR_CUDA;
     if (sync_check_enabled()) return fle_device_status(stream);
+    return FLE_OK;
+}
+
+int fle_plan_units(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int num_sms, int cta,
+                   int32_t* units, int max_units, int* n_units, int* grid) {
+    int st = check_desc(d);
+    if (st != FLE_OK) return st;
+    st = check_shape(M, K, N, d);
+    if (st != FLE_OK) return st;
+    if (num_sms <= 0 || cta < 0 || !n_units || (max_units > 0 && !units)) return FLE_ERR_NULL;
+    *n_units = 0;
+    if (grid) *grid = 0;
+    if (M == 0 || N == 0 || K == 0) return FLE_OK;
+    const Plan pl = make_plan(M, K, N, d, num_sms);
+    if (grid) *grid = pl.grid;
+    if (cta >= pl.grid) return FLE_OK;
+    KParams p{};
+    p.tiles_a = pl.tiles_a;
+    p.tiles_b = pl.tiles_b;
+    p.num_kb = pl.num_kb;
+    p.num_tiles = pl.tiles;
+    p.dp_tiles = pl.dp_tiles;
+    p.sk_iters = pl.sk_iters;
+    fle::Sched sc;
+    sc.init(p, cta, pl.grid);
+    fle::Unit u;
+    int n = 0;
+    while (sc.next(p, u)) {
+        if (n < max_units) {
+            int32_t* row = units + static_cast<size_t>(n) * 10;
+            row[0] = u.t; row[1] = u.ta; row[2] = u.tb; row[3] = u.kb0; row[4] = u.kb1;
+            row[5] = u.partial; row[6] = u.partial ? u.slot : -1;
+            if (u.partial) {
+                row[7] = fle::sk_cta_of(static_cast<int64_t>(u.sk_tile) * p.num_kb, p.sk_iters, pl.grid);
+                row[8] = fle::sk_cta_of((static_cast<int64_t>(u.sk_tile) + 1) * p.num_kb - 1, p.sk_iters, pl.grid);
+                row[9] = fle::sk_slot_of(cta, u.sk_tile, p.sk_iters, pl.grid, p.num_kb);
+            } else {
+                row[7] = row[8] = row[9] = -1;
+            }
+        }
+        ++n;
+    }
+    *n_units = n;
     return FLE_OK;
 }
 

@@ -1,8 +1,15 @@
 // fle_kernel.cuh -- the fused Linear + epilogue kernel for sm_100a.
 //
 // One persistent CTA per SM walks a list of work units.  A unit is one output
-// tile (128 rows of operand A x BN rows of operand B) over one range of
-// k-blocks (the whole K unless split-K is on).  Operand A is x and B is W
+// tile (128 rows of operand A x BN rows of operand B) over a range of
+// k-blocks.  The schedule is hybrid: the first whole waves of tiles are
+// data-parallel (one CTA per tile, the whole K), and the remaining tiles'
+// k-blocks are divided evenly over all CTAs (stream-K), so every SM gets the
+// same number of k-blocks whatever the tile count.  A tile whose k-range is
+// shared by several CTAs is finished by the last of them to arrive: each
+// writes its fp32 partial tile to the caller's workspace, and the last one sums
+// all partials in a fixed order (so results are bitwise reproducible) and
+// applies the epilogue.  Operand A is x and B is W
 // ("direct"), or, for small M, A is W and B is x ("swapped"), so the large
 // dimension sits on the 128-row side of the MMA; either way both operands are
 // K-major, as nn.Linear stores them.
@@ -42,14 +49,15 @@ enum : unsigned {
 struct KParams {
     const float* bias;      // [N] or nullptr
     float* out;             // [M,N] or [M]
-    float* ws;              // split-K partial tiles (nullptr when splits == 1)
-    unsigned* counters;     // split-K per-tile arrival counters
+    float* ws;              // stream-K partial tiles: [2 * grid][kBM * BN]
+    unsigned* counters;     // stream-K arrival counters, one per stream-K tile
     int64_t M, N;           // output sizes
     int Ma, Nb;             // rows of operand A and operand B
     int tiles_a, tiles_b;   // tiles along A rows and along B rows
     int num_kb;             // k-blocks along K
-    int splits, kb_per_split;
-    int num_units;
+    int num_tiles;          // tiles_a * tiles_b
+    int dp_tiles;           // tiles [0, dp_tiles) are data-parallel
+    int64_t sk_iters;       // (num_tiles - dp_tiles) * num_kb
     int kind;
     float scale, clamp_lo, clamp_hi;
     int pool_k;
@@ -58,6 +66,70 @@ struct KParams {
     int vec_bias;           // bias 16-byte aligned
     uint64_t timeout_ns;
 };
+
+// One unit of work: tile t over k-blocks [kb0, kb1).
+struct Unit {
+    int t, ta, tb;
+    int kb0, kb1;
+    int partial;            // the tile's k-range is shared with other CTAs
+    int sk_tile;            // index among the stream-K tiles
+    int slot;               // 0: first tile of this CTA's stream-K range, 1: last
+};
+
+// The unit sequence of one CTA.  Every role of the CTA walks it in lockstep.
+struct Sched {
+    int c, G;
+    int dp_next;
+    int64_t g, g_begin, g_end;
+
+    __host__ __device__ __forceinline__ void init(const KParams& p, int cta, int grid) {
+        c = cta;
+        G = grid;
+        dp_next = c;
+        g_begin = (static_cast<int64_t>(c) * p.sk_iters) / G;
+        g_end = (static_cast<int64_t>(c + 1) * p.sk_iters) / G;
+        g = g_begin;
+    }
+    __host__ __device__ __forceinline__ bool next(const KParams& p, Unit& u) {
+        if (dp_next < p.dp_tiles) {
+            u.t = dp_next;
+            u.kb0 = 0;
+            u.kb1 = p.num_kb;
+            u.partial = 0;
+            u.sk_tile = -1;
+            u.slot = 0;
+            dp_next += G;
+        } else if (g < g_end) {
+            const int64_t tsk = g / p.num_kb;
+            const int kb0 = static_cast<int>(g - tsk * p.num_kb);
+            const int64_t left = g_end - g;
+            const int kb1 = static_cast<int>(left < p.num_kb - kb0 ? kb0 + left : p.num_kb);
+            u.t = p.dp_tiles + static_cast<int>(tsk);
+            u.kb0 = kb0;
+            u.kb1 = kb1;
+            u.partial = (kb0 != 0 || kb1 != p.num_kb) ? 1 : 0;
+            u.sk_tile = static_cast<int>(tsk);
+            u.slot = (tsk == g_begin / p.num_kb) ? 0 : 1;
+            g += kb1 - kb0;
+        } else {
+            return false;
+        }
+        u.ta = u.t % p.tiles_a;
+        u.tb = u.t / p.tiles_a;
+        return true;
+    }
+};
+
+// The CTA whose stream-K range holds global stream-K k-block g.
+__host__ __device__ __forceinline__ int sk_cta_of(int64_t g, int64_t sk_iters, int G) {
+    return static_cast<int>(((g + 1) * G - 1) / sk_iters);
+}
+
+// Which of CTA c's two partial slots holds stream-K tile tsk.
+__host__ __device__ __forceinline__ int sk_slot_of(int c, int64_t tsk, int64_t sk_iters, int G, int num_kb) {
+    const int64_t gb = (static_cast<int64_t>(c) * sk_iters) / G;
+    return (tsk == gb / num_kb) ? 0 : 1;
+}
 
 template <int BN, int PREC>
 struct Cfg {
@@ -71,7 +143,7 @@ struct Cfg {
                                     : (2 * BN <= 256) ? 256 : 512;
     // barriers: full, conv, empty per stage; accf, acce per buffer; drain
     static constexpr int kNumBars = 3 * kStages + 4 + 1;
-    static constexpr int kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + kNumBars * 8 + 16;
+    static constexpr int kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + kNumBars * 8 + 32;
     static_assert(kStages >= 2, "need at least two stages");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128 is a multiple of 16 in [16,256]");
     static_assert(kABytes % 1024 == 0 && kBBytes % 1024 == 0, "tiles must keep 1024-byte alignment");
@@ -178,6 +250,45 @@ __device__ __forceinline__ void epi_store_swapped(const KParams& p, int64_t n, i
     }
 }
 
+// Epilogue for one 32-column chunk c of a unit's tile, whose accumulator
+// values (row r of the tile) are in v.  For the pool kind the chunk's complete
+// windows are folded into `best`; epi_finish then combines it across CTAs.
+template <bool SWAP, int BN>
+__device__ __forceinline__ void epi_chunk(const KParams& p, const Unit& u, int r, int c, float (&v)[32],
+                                          float& best) {
+    if constexpr (!SWAP) {
+        const int64_t m = static_cast<int64_t>(u.ta) * kBM + r;
+        const int64_t n0 = static_cast<int64_t>(u.tb) * BN + c * 32;
+        switch (p.kind) {
+            case kEpiHardtanhGelu: epi_store_direct<kEpiHardtanhGelu>(p, m, n0, v); break;
+            case kEpiSwish: epi_store_direct<kEpiSwish>(p, m, n0, v); break;
+            case kEpiPoolMax: epi_pool_direct(p, n0, v, best); break;
+            default: epi_store_direct<kEpiNone>(p, m, n0, v); break;
+        }
+    } else {
+        const int64_t n = static_cast<int64_t>(u.ta) * kBM + r;
+        const int64_t m0 = static_cast<int64_t>(u.tb) * BN + c * 32;
+        switch (p.kind) {
+            case kEpiHardtanhGelu: epi_store_swapped<kEpiHardtanhGelu>(p, n, m0, v); break;
+            case kEpiSwish: epi_store_swapped<kEpiSwish>(p, n, m0, v); break;
+            default: epi_store_swapped<kEpiNone>(p, n, m0, v); break;
+        }
+    }
+}
+
+template <bool SWAP>
+__device__ __forceinline__ void epi_finish(const KParams& p, const Unit& u, int r, float best) {
+    if constexpr (!SWAP) {
+        const int64_t m = static_cast<int64_t>(u.ta) * kBM + r;
+        if (p.kind == kEpiPoolMax && m < p.M && best > -INFINITY) atomic_max_f32(p.out + m, best);
+    }
+}
+
+// Barrier among the four epilogue warps only (named barrier 1, 128 threads).
+__device__ __forceinline__ void epilogue_bar_sync() {
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
 // ----------------------------------------------------------------------------
 // The kernel
 // ----------------------------------------------------------------------------
@@ -188,6 +299,8 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     using C = Cfg<BN, PREC>;
     constexpr int S = C::kStages;
     constexpr uint32_t kIdesc = idesc_tf32(kBM, BN);
+    // k-blocks per TMEM accumulation chain (see the epilogue role)
+    constexpr int kChunkKb = (PREC == kPrec3xTF32) ? 4 : (1 << 30);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -195,6 +308,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
     auto bar_full = [&](int s) { return smem_u32(bars + s); };
     auto bar_conv = [&](int s) { return smem_u32(bars + S + s); };
@@ -241,22 +355,19 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             uint32_t phase = 0;
             long long fills = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
-                const int ta = u % p.tiles_a;
-                const int rest = u / p.tiles_a;
-                const int tb = rest % p.tiles_b;
-                const int sp = rest / p.tiles_b;
-                const int kb0 = sp * p.kb_per_split;
-                const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
-                for (int kb = kb0; kb < kb1; ++kb) {
+            Sched sc;
+            sc.init(p, blockIdx.x, gridDim.x);
+            Unit u;
+            while (ok && sc.next(p, u)) {
+                for (int kb = u.kb0; kb < u.kb1; ++kb) {
                     if (!mbar_wait_bounded(bar_empty(stage), phase ^ 1u, abort_flag, p.timeout_ns,
                                            kWhereProdEmpty)) {
                         ok = false;
                         break;
                     }
                     mbar_arrive_expect_tx(bar_full(stage), C::kLoadBytes);
-                    tma_load_2d(sA(stage), &tmA, bar_full(stage), kb * kBK, ta * kBM);
-                    tma_load_2d(sB(stage), &tmB, bar_full(stage), kb * kBK, tb * BN);
+                    tma_load_2d(sA(stage), &tmA, bar_full(stage), kb * kBK, u.ta * kBM);
+                    tma_load_2d(sB(stage), &tmB, bar_full(stage), kb * kBK, u.tb * BN);
                     ++fills;
                     if (++stage == S) { stage = 0; phase ^= 1u; }
                 }
@@ -277,11 +388,13 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             int buf = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
-                const int rest = u / p.tiles_a;
-                const int sp = rest / p.tiles_b;
-                const int kb0 = sp * p.kb_per_split;
-                const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+            Sched sc;
+            sc.init(p, blockIdx.x, gridDim.x);
+            Unit u;
+            while (ok && sc.next(p, u)) {
+              // one accumulation chain per chunk of k-blocks (3xTF32) or per unit (TF32)
+              for (int kc = u.kb0; ok && kc < u.kb1; kc += kChunkKb) {
+                const int kce = (u.kb1 - kc > kChunkKb) ? kc + kChunkKb : u.kb1;
                 if (!mbar_wait_bounded(bar_acce(buf), acc_phase ^ 1u, abort_flag, p.timeout_ns,
                                        kWhereMmaAccEmpty)) {
                     ok = false;
@@ -289,7 +402,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 }
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
-                for (int kb = kb0; kb < kb1; ++kb) {
+                for (int kb = kc; kb < kce; ++kb) {
                     const uint32_t wbar = (PREC == kPrec3xTF32) ? bar_conv(stage) : bar_full(stage);
                     if (!mbar_wait_bounded(wbar, phase, abort_flag, p.timeout_ns, kWhereMmaFull)) {
                         ok = false;
@@ -302,7 +415,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     for (int k = 0; k < kBK / kUmmaK; ++k) {
                         // advance 8 fp32 = 32 bytes along K inside the swizzle atom
                         const uint64_t koff = static_cast<uint64_t>(k * 2);
-                        const uint32_t acc = (kb > kb0 || k > 0) ? 1u : 0u;
+                        const uint32_t acc = (kb > kc || k > 0) ? 1u : 0u;
                         if constexpr (PREC == kPrec3xTF32) {
                             const uint64_t a_lo = smem_desc_sw128(sA(stage) + C::kLoadBytes);
                             const uint64_t b_lo = smem_desc_sw128(sB(stage) + C::kLoadBytes);
@@ -320,6 +433,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 mma_commit(bar_accf(buf));
                 buf ^= 1;
                 if (buf == 0) acc_phase ^= 1u;
+              }
             }
             // All issued MMAs must be complete before TMEM is released.
             mma_commit(bar_drain);
@@ -334,12 +448,11 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
-                const int rest = u / p.tiles_a;
-                const int sp = rest / p.tiles_b;
-                const int kb0 = sp * p.kb_per_split;
-                const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
-                for (int kb = kb0; kb < kb1; ++kb) {
+            Sched sc;
+            sc.init(p, blockIdx.x, gridDim.x);
+            Unit u;
+            while (ok && sc.next(p, u)) {
+                for (int kb = u.kb0; kb < u.kb1; ++kb) {
                     int got = 0;
                     if (lane == 0)
                         got = mbar_wait_bounded(bar_full(stage), phase, abort_flag, p.timeout_ns, kWhereConvFull);
@@ -371,55 +484,154 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int q = warp - 4;  // TMEM lane quadrant of this warp
+        const int q = warp - 4;       // TMEM lane quadrant of this warp
+        const int r = q * 32 + lane;  // tile row = TMEM lane of this thread
         int buf = 0;
         uint32_t acc_phase = 0;
-        for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
-            const int ta = u % p.tiles_a;
-            const int rest = u / p.tiles_a;
-            const int tb = rest % p.tiles_b;
-            int got = 0;
-            if (lane == 0)
-                got = mbar_wait_bounded(bar_accf(buf), acc_phase, abort_flag, p.timeout_ns, kWhereEpiAccFull);
-            got = __shfl_sync(0xffffffffu, got, 0);
-            if (!got) break;
-            tc_fence_after_sync();
-            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * BN);
-            if constexpr (!SWAP) {
-                const int64_t m = static_cast<int64_t>(ta) * kBM + q * 32 + lane;
-                float best = -INFINITY;
-                for (int c = 0; c < BN / 32; ++c) {
-                    const int64_t n0 = static_cast<int64_t>(tb) * BN + c * 32;
-                    if (n0 >= p.N) break;  // warp-uniform
-                    float v[32];
-                    tmem_ld32_wait(t_row + c * 32, v);
-                    switch (p.kind) {
-                        case kEpiHardtanhGelu: epi_store_direct<kEpiHardtanhGelu>(p, m, n0, v); break;
-                        case kEpiSwish: epi_store_direct<kEpiSwish>(p, m, n0, v); break;
-                        case kEpiPoolMax: epi_pool_direct(p, n0, v, best); break;
-                        default: epi_store_direct<kEpiNone>(p, m, n0, v); break;
+        // 3xTF32 accumulates each kChunkKb-deep slice of K in a fresh TMEM
+        // buffer and sums the slices here, in fp32 registers with
+        // round-to-nearest: the tensor core's own accumulation rounds toward
+        // zero, whose bias would otherwise grow with the length of K.
+        constexpr bool kRegAcc = (PREC == kPrec3xTF32);
+        float accr[kRegAcc ? BN : 1];
+        Sched sc;
+        sc.init(p, blockIdx.x, gridDim.x);
+        Unit u;
+        bool ok = true;
+        while (ok && sc.next(p, u)) {
+            // 32-column chunks of this tile that hold any output (warp-uniform)
+            const int64_t cols_left = (SWAP ? p.M : p.N) - static_cast<int64_t>(u.tb) * BN;
+            const int nchunks = static_cast<int>(cols_left >= BN ? BN / 32 : (cols_left + 31) / 32);
+
+            auto wait_acc = [&]() -> bool {
+                int got = 0;
+                if (lane == 0)
+                    got = mbar_wait_bounded(bar_accf(buf), acc_phase, abort_flag, p.timeout_ns, kWhereEpiAccFull);
+                got = __shfl_sync(0xffffffffu, got, 0);
+                if (got) tc_fence_after_sync();
+                return got != 0;
+            };
+            auto release_acc = [&]() {
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_acce(buf));
+                buf ^= 1;
+                if (buf == 0) acc_phase ^= 1u;
+            };
+            auto t_row = [&]() {
+                return tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * BN);
+            };
+
+            uint32_t t_acc = 0;
+            if constexpr (kRegAcc) {
+#pragma unroll
+                for (int j = 0; j < (kRegAcc ? BN : 1); ++j) accr[j] = 0.0f;
+                for (int kc = u.kb0; kc < u.kb1; kc += kChunkKb) {
+                    if (!wait_acc()) { ok = false; break; }
+                    const uint32_t tr = t_row();
+#pragma unroll
+                    for (int c = 0; c < BN / 32; ++c) {
+                        if (c >= nchunks) break;
+                        float v[32];
+                        tmem_ld32_wait(tr + c * 32, v);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) accr[c * 32 + j] += v[j];
                     }
+                    release_acc();
                 }
-                if (p.kind == kEpiPoolMax && m < p.M && best > -INFINITY) atomic_max_f32(p.out + m, best);
+                if (!ok) break;
             } else {
-                const int64_t n = static_cast<int64_t>(ta) * kBM + q * 32 + lane;
-                for (int c = 0; c < BN / 32; ++c) {
-                    const int64_t m0 = static_cast<int64_t>(tb) * BN + c * 32;
-                    if (m0 >= p.M) break;  // warp-uniform
-                    float v[32];
-                    tmem_ld32_wait(t_row + c * 32, v);
-                    switch (p.kind) {
-                        case kEpiHardtanhGelu: epi_store_swapped<kEpiHardtanhGelu>(p, n, m0, v); break;
-                        case kEpiSwish: epi_store_swapped<kEpiSwish>(p, n, m0, v); break;
-                        default: epi_store_swapped<kEpiNone>(p, n, m0, v); break;
+                if (!wait_acc()) break;
+                t_acc = t_row();
+            }
+            // The 32 accumulator values of chunk c of this unit, in registers
+            // (3xTF32) or in TMEM (TF32).  Called with compile-time c when the
+            // values are registers.
+#define FLE_LOAD_ACC(c, v)                                                        \
+    do {                                                                          \
+        if constexpr (kRegAcc) {                                                  \
+            _Pragma("unroll") for (int j_ = 0; j_ < 32; ++j_) v[j_] = accr[(c) * 32 + j_]; \
+        } else {                                                                  \
+            tmem_ld32_wait(t_acc + (c) * 32, v);                                  \
+        }                                                                         \
+    } while (0)
+
+            if (!u.partial) {
+                float best = -INFINITY;
+#define FLE_EPI_BODY(c)                          \
+    {                                            \
+        float v[32];                             \
+        FLE_LOAD_ACC(c, v);                      \
+        epi_chunk<SWAP, BN>(p, u, r, c, v, best); \
+    }
+                if constexpr (kRegAcc) {
+#pragma unroll
+                    for (int c = 0; c < BN / 32; ++c)
+                        if (c < nchunks) FLE_EPI_BODY(c)
+                } else {
+#pragma unroll 1
+                    for (int c = 0; c < nchunks; ++c) FLE_EPI_BODY(c)
+                }
+#undef FLE_EPI_BODY
+                epi_finish<SWAP>(p, u, r, best);
+                if constexpr (!kRegAcc) release_acc();
+            } else {
+                // Park this CTA's fp32 partial tile in its workspace slot.
+                float* mine = p.ws + (static_cast<size_t>(2 * blockIdx.x + u.slot) * kBM + r) * BN;
+#define FLE_PARK_BODY(c)                                                                            \
+    {                                                                                               \
+        float v[32];                                                                                \
+        FLE_LOAD_ACC(c, v);                                                                         \
+        float4* d4 = reinterpret_cast<float4*>(mine + (c) * 32);                                    \
+        _Pragma("unroll") for (int j = 0; j < 8; ++j)                                               \
+            __stcg(d4 + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));        \
+    }
+                if constexpr (kRegAcc) {
+#pragma unroll
+                    for (int c = 0; c < BN / 32; ++c)
+                        if (c < nchunks) FLE_PARK_BODY(c)
+                } else {
+#pragma unroll 1
+                    for (int c = 0; c < nchunks; ++c) FLE_PARK_BODY(c)
+                }
+#undef FLE_PARK_BODY
+                if constexpr (!kRegAcc) release_acc();
+                const int64_t tsk = u.sk_tile;
+                const int first = sk_cta_of(tsk * p.num_kb, p.sk_iters, gridDim.x);
+                const int last = sk_cta_of((tsk + 1) * p.num_kb - 1, p.sk_iters, gridDim.x);
+                __threadfence();
+                epilogue_bar_sync();
+                if (threadIdx.x == 128) {
+                    const unsigned prev = atomicAdd(p.counters + tsk, 1u);
+                    *last_flag = (prev == static_cast<unsigned>(last - first)) ? 1 : 0;
+                }
+                epilogue_bar_sync();
+                if (*last_flag) {
+                    // Last to arrive: sum every contributor's partial in CTA
+                    // order (= k order), then run the epilogue on the sum.
+                    __threadfence();
+                    float best = -INFINITY;
+                    for (int c = 0; c < nchunks; ++c) {
+                        float v[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+                        for (int cc = first; cc <= last; ++cc) {
+                            const int sl = sk_slot_of(cc, tsk, p.sk_iters, gridDim.x, p.num_kb);
+                            const float4* s4 = reinterpret_cast<const float4*>(
+                                p.ws + (static_cast<size_t>(2 * cc + sl) * kBM + r) * BN + c * 32);
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const float4 t = __ldcg(s4 + j);
+                                v[4 * j] += t.x; v[4 * j + 1] += t.y; v[4 * j + 2] += t.z; v[4 * j + 3] += t.w;
+                            }
+                        }
+                        epi_chunk<SWAP, BN>(p, u, r, c, v, best);
                     }
+                    epi_finish<SWAP>(p, u, r, best);
+                    if (threadIdx.x == 128) p.counters[tsk] = 0u;
                 }
             }
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_acce(buf));
-            buf ^= 1;
-            if (buf == 0) acc_phase ^= 1u;
+#undef FLE_LOAD_ACC
         }
     }
 
@@ -457,9 +669,13 @@ __global__ void fle_bias_only_kernel(const KParams p) {
     p.out[i] = o;
 }
 
-__global__ void fle_fill_kernel(float* out, int64_t n, float v) {
+// Per-call preparation on the caller's stream: out[M] = -inf for the pool
+// kind (the row maximum is combined with atomics) and zeroed stream-K
+// arrival counters.
+__global__ void fle_prep_kernel(float* fill, int64_t n_fill, unsigned* counters, int n_counters) {
     const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (i < n) out[i] = v;
+    if (fill != nullptr && i < n_fill) fill[i] = -INFINITY;
+    if (counters != nullptr && i < n_counters) counters[i] = 0u;
 }
 
 // Test hook: one thread waits on a barrier nothing arrives on.

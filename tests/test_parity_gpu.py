@@ -241,3 +241,33 @@ def test_tf32_input_conversion_probe(fle, capsys):
     assert got in (trunc, rn), got
     with capsys.disabled():
         print(f"\n[tf32 operand conversion: {'truncate' if got == trunc else 'round-to-nearest'}]")
+
+
+def test_tensor_core_accumulation_rounding_probe(fle, capsys):
+    # One tile, 15 k-blocks (too few to be split across CTAs): x = 1, W[0,0] = 1
+    # and every other W = 1.5 * 2^-27, so each 8-deep MMA after the first adds
+    # 0.75 ulp(1) to an accumulator of 1.0.  Truncating accumulation keeps 1.0;
+    # round-to-nearest climbs by one ulp per instruction; the exact sum is about
+    # 1 + 45 ulp.  Informational: the 3xTF32 path sums 128-deep slices in
+    # registers, which bounds the error whichever way the hardware rounds.
+    K = 15 * 32
+    x = torch.ones(1, K, device="cuda")
+    W = torch.full((1, K), 1.5 * 2.0 ** -27, device="cuda")
+    W[0, 0] = 1.0
+    out = _run(fle, x, W, None, "none", "tf32")
+    ulps = (float(out[0, 0]) - 1.0) / 2.0 ** -23
+    assert -0.5 <= ulps <= 61, ulps
+    mode = "truncating (round toward zero)" if ulps < 0.5 else f"{ulps:.0f} ulp above 1 (rounding)"
+    with capsys.disabled():
+        print(f"\n[tensor-core fp32 accumulation: {mode}]")
+
+
+@pytest.mark.parametrize("precision", ["3xtf32"])
+def test_long_k_accuracy_3xtf32(fle, precision):
+    # The accumulation chain grows with K; 3xTF32 must keep the fp32-faithful
+    # bound at K = 32768 on unit-scale data (direct and swapped order).
+    for M, N in ((128, 640), (300, 260)):
+        x, W, b = synth.linear_inputs(M, 32768, N, seed=M, device="cuda")
+        out = _run(fle, x, W, b, "none", precision)
+        rows = synth.sample_rows(M, 32, seed=2)
+        _assert_close(out.cpu().numpy()[rows], _oracle(x, W, b, "none", rows=rows), precision, f"K=32768 {M}x{N}")

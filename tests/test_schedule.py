@@ -1,0 +1,121 @@
+"""Host-side checks of the persistent schedule (no GPU needed).
+
+The kernel's work list comes from the same scheduler code that
+fle_plan_units runs on the host.  For every workload below, over all CTAs of
+the plan: each tile's k-blocks are computed exactly once; a tile computed
+whole has one unit; a shared (stream-K) tile's contributors are exactly the
+CTAs first..last that the finishing CTA will read, in k order, each with the
+workspace slot the finishing CTA expects; no CTA holds more than two shared
+tiles; and the k-blocks are balanced across CTAs.
+"""
+import math
+from collections import defaultdict
+
+import pytest
+
+import reduction_epilogue_b200 as fle
+from reduction_epilogue_b200 import build as fle_build
+
+WORKLOADS = [
+    (128, 1024, 1024, "scale_hardtanh_gelu"),
+    (2048, 8192, 8192, "scale_hardtanh_gelu"),
+    (1024, 8192, 8192, "avgpool_gelu_scale_rowmax"),
+    (128, 32768, 32768, "swish_scale"),
+    (16, 8192, 8192, "scale_hardtanh_gelu"),
+    (64, 8192, 8192, "scale_hardtanh_gelu"),
+    (256, 8192, 8192, "scale_hardtanh_gelu"),
+    (1024, 8192, 8192, "scale_hardtanh_gelu"),
+    (4096, 8192, 8192, "scale_hardtanh_gelu"),
+    (7, 36, 33, "swish_scale"),
+    (300, 132, 1000, "none"),
+    (129, 4100, 777, "none"),
+    (33, 20000, 3000, "scale_hardtanh_gelu"),
+]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    fle_build.build()
+    fle.load()
+
+
+def collect(M, K, N, desc, sms):
+    grid, _ = fle.plan_units(M, K, N, desc, sms, 0)
+    per_cta = [fle.plan_units(M, K, N, desc, sms, c)[1] for c in range(grid)]
+    return grid, per_cta
+
+
+@pytest.mark.parametrize("sms", [148, 132, 7])
+@pytest.mark.parametrize("precision", ["tf32", "3xtf32"])
+@pytest.mark.parametrize("M,K,N,problem", WORKLOADS)
+def test_schedule_covers_every_kblock_once(M, K, N, problem, precision, sms):
+    desc = fle.desc_for(problem, precision)
+    grid, per_cta = collect(M, K, N, desc, sms)
+    assert 1 <= grid <= sms
+    num_kb = math.ceil(K / 32)
+    cover = defaultdict(list)  # tile -> [(kb0, kb1, cta, row)]
+    for c, rows in enumerate(per_cta):
+        partial_slots = []
+        for r in rows:
+            t, ta, tb, kb0, kb1, partial, slot, first, last, slot_rule = (int(v) for v in r)
+            assert 0 <= kb0 < kb1 <= num_kb
+            cover[t].append((kb0, kb1, c, (ta, tb), partial, slot, first, last, slot_rule))
+            if partial:
+                partial_slots.append(slot)
+                assert slot == slot_rule
+        assert len(partial_slots) <= 2 and len(set(partial_slots)) == len(partial_slots)
+
+    tiles = sorted(cover)
+    assert tiles == list(range(len(tiles)))
+    tas = {e[3][0] for v in cover.values() for e in v}
+    tbs = {e[3][1] for v in cover.values() for e in v}
+    assert len(tas) * len(tbs) == len(tiles)
+    # the tiles span exactly the operand rows (A side holds M or N)
+    a_rows = {math.ceil(M / 128), math.ceil(N / 128)}
+    assert len(tas) in a_rows
+
+    for t, units in cover.items():
+        units.sort()
+        # exact cover of [0, num_kb)
+        pos = 0
+        for kb0, kb1, *_ in units:
+            assert kb0 == pos
+            pos = kb1
+        assert pos == num_kb
+        assert len({u[3] for u in units}) == 1  # one (ta, tb) per tile
+        if len(units) == 1:
+            assert units[0][4] == 0  # whole tile, not shared
+        else:
+            ctas = [u[2] for u in units]
+            assert all(u[4] == 1 for u in units)
+            first, last = units[0][6], units[0][7]
+            assert all((u[6], u[7]) == (first, last) for u in units)
+            assert ctas == list(range(first, last + 1))  # CTA order = k order
+
+    # balance: stream-K spreads the remainder evenly
+    load = [sum(int(r[4]) - int(r[3]) for r in rows) for rows in per_cta]
+    assert sum(load) == len(tiles) * num_kb
+    assert max(load) - min(load) <= num_kb
+
+
+def test_headline_shape_is_balanced_to_one_kblock():
+    # 2048x8192x8192 with 128x256 tiles: 512 tiles on 148 SMs is 3.46 waves;
+    # the hybrid schedule gives every SM the same k-block count to within one.
+    desc = fle.desc_for("scale_hardtanh_gelu", "tf32")
+    grid, per_cta = collect(2048, 8192, 8192, desc, 148)
+    assert grid == 148
+    load = [sum(int(r[4]) - int(r[3]) for r in rows) for rows in per_cta]
+    assert max(load) - min(load) <= 1
+    assert sum(load) == 512 * 256
+
+
+def test_workspace_matches_the_plan():
+    # two fp32 partial tiles per CTA plus one counter per shared tile
+    desc = fle.desc_for("swish_scale", "tf32")
+    lib = fle.load()
+    import ctypes
+    n = ctypes.c_int(0)
+    g = ctypes.c_int(0)
+    assert lib.fle_plan_units(128, 32768, 32768, ctypes.byref(desc), 148, 0, None, 0,
+                              ctypes.byref(n), ctypes.byref(g)) == 0
+    assert g.value == 148
