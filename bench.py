@@ -366,6 +366,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(CONFIGS))
     ap.add_argument("--all", action="store_true", help="one line per config")
+    ap.add_argument("--shape", default=None,
+                    help="M,K,N,problem: a custom workload (for profiling smaller cases)")
     ap.add_argument("--precision", default="tf32", choices=["tf32", "3xtf32"])
     ap.add_argument("--impl", default="fle", choices=["fle", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
@@ -376,6 +378,11 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     names = sorted(CONFIGS) if args.all else [args.config]
+    if args.shape:
+        M, K, N, problem = args.shape.split(",")
+        name = f"custom_m{M}_k{K}_n{N}_{problem}"
+        CONFIGS[name] = (int(M), int(K), int(N), problem)
+        names = [name]
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

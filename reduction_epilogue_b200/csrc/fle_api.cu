@@ -104,8 +104,9 @@ struct Plan {
     int tiles_a = 0, tiles_b = 0, tiles = 0;
     int num_kb = 0;
     int dp_tiles = 0;          // tiles done whole, one CTA each
-    int64_t sk_iters = 0;      // k-blocks of the remaining tiles, spread over the grid
+    int64_t sk_iters = 0;      // k-blocks of the remaining tiles, spread over sk_grid CTAs
     int sk_tiles = 0;
+    int sk_grid = 0;
     int grid = 0;
     size_t partial_bytes = 0;  // workspace: 2 partial tiles per CTA ...
     size_t ws_bytes = 0;       // ... then one arrival counter per stream-K tile
@@ -148,27 +149,39 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
     const int64_t T = pl.tiles;
     const int64_t G = sms;
     const int64_t iters = T * pl.num_kb;
-    const bool force_dp = std::strcmp(sched_override(), "dp") == 0;
+    // Is a weight tile used by more than one tile of the output?  Then CTAs
+    // sharing it must walk K in step to reuse it from L2.
+    const bool w_shared = (pl.swap ? pl.tiles_b : pl.tiles_a) > 1;
+    const char* ov = sched_override();
+    const bool force_dp = std::strcmp(ov, "dp") == 0;
     pl.dp_tiles = static_cast<int>(T);
     pl.grid = static_cast<int>(T < G ? T : G);
-    if (!force_dp && T % G != 0 && pl.num_kb >= kMinSkIters) {
-        if (T > G) {
-            // keep all but the last full wave data-parallel; the last full wave
-            // plus the partial one are spread evenly over every CTA
-            pl.dp_tiles = static_cast<int>((T / G - 1) * G);
-            pl.grid = static_cast<int>(G);
-        } else {
+    pl.sk_grid = 0;
+    if (!force_dp && T % G != 0 && pl.num_kb >= 2 * kMinSkIters) {
+        if (!w_shared && T < G) {
+            // every weight tile is read by one unit: spread all k-blocks over the SMs
             const int64_t g_sk = std::min<int64_t>(G, iters / kMinSkIters);
             if (g_sk > T) {
                 pl.dp_tiles = 0;
                 pl.grid = static_cast<int>(g_sk);
+                pl.sk_grid = pl.grid;
+            }
+        } else {
+            // full waves data-parallel; the R tiles of the last partial wave
+            // split into S k-aligned parts on R*S CTAs
+            const int64_t R = T % G;
+            const int64_t S = std::min<int64_t>(G / R, pl.num_kb / kMinSkIters);
+            if (S >= 2) {
+                pl.dp_tiles = static_cast<int>(T - R);
+                pl.grid = static_cast<int>(T > G ? G : R * S);
+                pl.sk_grid = static_cast<int>(R * S);
             }
         }
     }
     pl.sk_tiles = static_cast<int>(T - pl.dp_tiles);
     pl.sk_iters = static_cast<int64_t>(pl.sk_tiles) * pl.num_kb;
     if (pl.sk_tiles > 0) {
-        pl.partial_bytes = static_cast<size_t>(2) * pl.grid * fle::kBM * pl.bn * sizeof(float);
+        pl.partial_bytes = static_cast<size_t>(2) * pl.sk_grid * fle::kBM * pl.bn * sizeof(float);
         pl.ws_bytes = pl.partial_bytes + ((static_cast<size_t>(pl.sk_tiles) * 4 + 255) & ~size_t(255));
     }
     return pl;
@@ -243,9 +256,9 @@ int plan_to_string(const Plan& pl, char* buf, size_t n) {
     if (!buf || n == 0) return FLE_ERR_NULL;
     std::snprintf(buf, n,
                   "tile=128x%d swap=%d prec=%s stages=%d tiles=%dx%d kblocks=%d dp_tiles=%d sk_tiles=%d "
-                  "sk_kblocks=%lld grid=%d workspace=%zu",
+                  "sk_kblocks=%lld sk_grid=%d grid=%d workspace=%zu",
                   pl.bn, pl.swap ? 1 : 0, pl.prec == fle::kPrecTF32 ? "tf32" : "3xtf32", pl.stages,
-                  pl.tiles_a, pl.tiles_b, pl.num_kb, pl.dp_tiles, pl.sk_tiles, (long long)pl.sk_iters, pl.grid,
+                  pl.tiles_a, pl.tiles_b, pl.num_kb, pl.dp_tiles, pl.sk_tiles, (long long)pl.sk_iters, pl.sk_grid, pl.grid,
                   pl.ws_bytes);
     return FLE_OK;
 }
@@ -348,6 +361,7 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
     p.num_tiles = pl.tiles;
     p.dp_tiles = pl.dp_tiles;
     p.sk_iters = pl.sk_iters;
+    p.sk_grid = pl.sk_grid;
     if (pl.sk_tiles > 0) {
         p.ws = static_cast<float*>(workspace);
         p.counters = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + pl.partial_bytes);
@@ -400,6 +414,7 @@ int fle_plan_units(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, 
     p.num_tiles = pl.tiles;
     p.dp_tiles = pl.dp_tiles;
     p.sk_iters = pl.sk_iters;
+    p.sk_grid = pl.sk_grid;
     fle::Sched sc;
     sc.init(p, cta, pl.grid);
     fle::Unit u;
@@ -410,9 +425,9 @@ int fle_plan_units(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, 
             row[0] = u.t; row[1] = u.ta; row[2] = u.tb; row[3] = u.kb0; row[4] = u.kb1;
             row[5] = u.partial; row[6] = u.partial ? u.slot : -1;
             if (u.partial) {
-                row[7] = fle::sk_cta_of(static_cast<int64_t>(u.sk_tile) * p.num_kb, p.sk_iters, pl.grid);
-                row[8] = fle::sk_cta_of((static_cast<int64_t>(u.sk_tile) + 1) * p.num_kb - 1, p.sk_iters, pl.grid);
-                row[9] = fle::sk_slot_of(cta, u.sk_tile, p.sk_iters, pl.grid, p.num_kb);
+                row[7] = fle::sk_cta_of(static_cast<int64_t>(u.sk_tile) * p.num_kb, p.sk_iters, pl.sk_grid);
+                row[8] = fle::sk_cta_of((static_cast<int64_t>(u.sk_tile) + 1) * p.num_kb - 1, p.sk_iters, pl.sk_grid);
+                row[9] = fle::sk_slot_of(cta, u.sk_tile, p.sk_iters, pl.sk_grid, p.num_kb);
             } else {
                 row[7] = row[8] = row[9] = -1;
             }

@@ -2,10 +2,14 @@
 //
 // One persistent CTA per SM walks a list of work units.  A unit is one output
 // tile (128 rows of operand A x BN rows of operand B) over a range of
-// k-blocks.  The schedule is hybrid: the first whole waves of tiles are
-// data-parallel (one CTA per tile, the whole K), and the remaining tiles'
-// k-blocks are divided evenly over all CTAs (stream-K), so every SM gets the
-// same number of k-blocks whatever the tile count.  A tile whose k-range is
+// k-blocks.  The schedule is hybrid: the first tiles are data-parallel (one
+// CTA per tile, the whole K), and the remaining tiles' k-blocks are divided
+// evenly over the first sk_grid CTAs (stream-K), so the SMs get equal shares
+// of k-blocks whatever the tile count.  The host picks the split (see
+// make_plan): shapes that stream each weight tile once spread the stream-K
+// part over every SM; shapes whose weight tiles are shared by several tiles
+// split only the last partial wave, into k-aligned parts, so the CTAs that
+// share a weight slab still walk K together and hit it in L2.  A tile whose k-range is
 // shared by several CTAs is finished by the last of them to arrive: each
 // writes its fp32 partial tile to the caller's workspace, and the last one sums
 // all partials in a fixed order (so results are bitwise reproducible) and
@@ -58,6 +62,7 @@ struct KParams {
     int num_tiles;          // tiles_a * tiles_b
     int dp_tiles;           // tiles [0, dp_tiles) are data-parallel
     int64_t sk_iters;       // (num_tiles - dp_tiles) * num_kb
+    int sk_grid;            // CTAs [0, sk_grid) share the stream-K k-blocks
     int kind;
     float scale, clamp_lo, clamp_hi;
     int pool_k;
@@ -86,8 +91,12 @@ struct Sched {
         c = cta;
         G = grid;
         dp_next = c;
-        g_begin = (static_cast<int64_t>(c) * p.sk_iters) / G;
-        g_end = (static_cast<int64_t>(c + 1) * p.sk_iters) / G;
+        if (c < p.sk_grid) {
+            g_begin = (static_cast<int64_t>(c) * p.sk_iters) / p.sk_grid;
+            g_end = (static_cast<int64_t>(c + 1) * p.sk_iters) / p.sk_grid;
+        } else {
+            g_begin = g_end = 0;
+        }
         g = g_begin;
     }
     __host__ __device__ __forceinline__ bool next(const KParams& p, Unit& u) {
@@ -120,7 +129,7 @@ struct Sched {
     }
 };
 
-// The CTA whose stream-K range holds global stream-K k-block g.
+// The CTA whose stream-K range holds global stream-K k-block g (G = sk_grid).
 __host__ __device__ __forceinline__ int sk_cta_of(int64_t g, int64_t sk_iters, int G) {
     return static_cast<int>(((g + 1) * G - 1) / sk_iters);
 }
@@ -597,8 +606,8 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 #undef FLE_PARK_BODY
                 if constexpr (!kRegAcc) release_acc();
                 const int64_t tsk = u.sk_tile;
-                const int first = sk_cta_of(tsk * p.num_kb, p.sk_iters, gridDim.x);
-                const int last = sk_cta_of((tsk + 1) * p.num_kb - 1, p.sk_iters, gridDim.x);
+                const int first = sk_cta_of(tsk * p.num_kb, p.sk_iters, p.sk_grid);
+                const int last = sk_cta_of((tsk + 1) * p.num_kb - 1, p.sk_iters, p.sk_grid);
                 __threadfence();
                 epilogue_bar_sync();
                 if (threadIdx.x == 128) {
@@ -616,7 +625,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 #pragma unroll
                         for (int j = 0; j < 32; ++j) v[j] = 0.0f;
                         for (int cc = first; cc <= last; ++cc) {
-                            const int sl = sk_slot_of(cc, tsk, p.sk_iters, gridDim.x, p.num_kb);
+                            const int sl = sk_slot_of(cc, tsk, p.sk_iters, p.sk_grid, p.num_kb);
                             const float4* s4 = reinterpret_cast<const float4*>(
                                 p.ws + (static_cast<size_t>(2 * cc + sl) * kBM + r) * BN + c * 32);
 #pragma unroll

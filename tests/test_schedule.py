@@ -98,15 +98,29 @@ def test_schedule_covers_every_kblock_once(M, K, N, problem, precision, sms):
     assert max(load) - min(load) <= num_kb
 
 
-def test_headline_shape_is_balanced_to_one_kblock():
-    # 2048x8192x8192 with 128x256 tiles: 512 tiles on 148 SMs is 3.46 waves;
-    # the hybrid schedule gives every SM the same k-block count to within one.
+def test_headline_shape_splits_only_the_last_wave():
+    # 2048x8192x8192 with 128x256 tiles: 512 tiles on 148 SMs is 3.46 waves.
+    # Three waves run whole tiles; the 68 tiles of the last wave are split in
+    # two k-aligned halves on 136 CTAs, so the SMs finish within half a tile.
     desc = fle.desc_for("scale_hardtanh_gelu", "tf32")
     grid, per_cta = collect(2048, 8192, 8192, desc, 148)
     assert grid == 148
     load = [sum(int(r[4]) - int(r[3]) for r in rows) for rows in per_cta]
-    assert max(load) - min(load) <= 1
     assert sum(load) == 512 * 256
+    assert max(load) - min(load) == 128
+    halves = [r for rows in per_cta for r in rows if r[5]]
+    assert len(halves) == 136
+    assert {(int(r[3]), int(r[4])) for r in halves} == {(0, 128), (128, 256)}
+
+
+def test_weight_streamed_once_shapes_use_every_sm():
+    # M = 16 (swapped): 64 weight tiles, each read by one unit; all 148 SMs
+    # share the k-blocks evenly (to within one).
+    desc = fle.desc_for("scale_hardtanh_gelu", "tf32")
+    grid, per_cta = collect(16, 8192, 8192, desc, 148)
+    assert grid == 148
+    load = [sum(int(r[4]) - int(r[3]) for r in rows) for rows in per_cta]
+    assert max(load) - min(load) <= 1
 
 
 def test_workspace_matches_the_plan():
