@@ -150,6 +150,36 @@ int fle_plan_string(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* de
 int fle_plan_units(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* desc, int num_sms,
                    int cta, int32_t* units, int max_units, int* n_units, int* grid);
 
+/*
+ * fle_forward_noalloc -- fle_forward without a caller workspace.
+ *
+ * (The pages have no counterpart of this call: it serves callers of this
+ * library, not the method.)  Some callers cannot allocate device memory at
+ * the point where they run the layer: a serving process that hands each
+ * model a fixed slice of HBM up front and forbids later allocations, or a
+ * latency-critical loop in which cudaMalloc/cudaFree would synchronise the
+ * device and stall every other stream.  This entry point needs no workspace
+ * argument and allocates nothing: the scratch that fle_forward takes from
+ * `workspace` (stream-K partial tiles and arrival counters) comes from one
+ * static device array of FLE_NOALLOC_SCRATCH_BYTES (40 MiB) inside the
+ * library.  Every plan on a 148-SM B200 needs at most about 37 MiB; a plan
+ * that would need more is rejected with FLE_ERR_WORKSPACE before anything is
+ * enqueued.  The caller still owns and passes x, W, b and out, with the same
+ * layout, alignment and error rules as fle_forward.
+ *
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture on
+ * the device.  Every GPU that loads the library keeps the array for the life
+ * of the process.  All calls on a device share the one array, and it keeps
+ * whatever the last call left in it; each call clears the counters it needs
+ * before use.  Calls whose kernels overlap on the GPU (other streams, other
+ * threads) race on the shared scratch and give wrong results: serialise them.
+ */
+#define FLE_NOALLOC_SCRATCH_BYTES ((size_t)40 << 20)
+int fle_forward_noalloc(const float* x, const float* W, const float* b,
+                        int64_t M, int64_t K, int64_t N,
+                        const fle_epilogue_desc* desc, float* out, void* stream);
+
 /* Library ABI version (major * 10000 + minor * 100 + patch). */
 int fle_version(void);
 

@@ -226,3 +226,26 @@ def linear_epilogue(x, W, b, problem: str = "scale_hardtanh_gelu", precision: st
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=x.device) if ws_bytes else None
     forward(x, W, b, out, desc, workspace=ws, workspace_bytes=ws_bytes, stream=stream)
     return out
+
+
+def forward_noalloc(x, W, b, out, desc: EpilogueDesc, stream=None) -> None:
+    """Calls fle_forward_noalloc: fle_forward with the library's own static
+    scratch instead of a caller workspace, for callers that cannot allocate
+    device memory where they run the layer.  Calls that overlap on the GPU
+    share that scratch and must be serialised."""
+    lib = load()
+    fn = lib.fle_forward_noalloc
+    vp = ctypes.c_void_p
+    fn.argtypes = [vp, vp, vp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                   ctypes.POINTER(EpilogueDesc), vp, vp]
+    fn.restype = ctypes.c_int
+    M, K = x.shape
+    N = W.shape[0]
+    _check_tensor("x", x, (M, K))
+    _check_tensor("W", W, (N, K))
+    _check_tensor("b", b, (N,))
+    _check_tensor("out", out, (M,) if desc.kind == EPI_AVGPOOL_GELU_SCALE_ROWMAX else (M, N))
+    st = fn(_ptr(x), _ptr(W), _ptr(b), int(M), int(K), int(N), ctypes.byref(desc), _ptr(out),
+            _stream_handle(stream))
+    if st != FLE_OK:
+        raise FleError(st, "fle_forward_noalloc")

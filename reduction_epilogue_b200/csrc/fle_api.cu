@@ -462,3 +462,42 @@ int fle_test_bounded_wait(uint32_t timeout_us, void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free entry point.  Its scratch (the stream-K partial tiles and
+// arrival counters that fle_forward takes from the caller's workspace) lives
+// in this file-scope device array instead, so the call needs no allocation
+// by anyone.  The array is part of the library's device image: every GPU
+// that loads the library holds these bytes until the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FLE_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch per device.  In host code the array's
+// name only stands in for the symbol; the address a kernel can use comes
+// from cudaGetSymbolAddress, taken with that device current.
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+}  // namespace
+
+extern "C" int fle_forward_noalloc(const float* x, const float* W, const float* b, int64_t M, int64_t K,
+                                   int64_t N, const fle_epilogue_desc* d, float* out, void* stream) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FLE_ERR_CUDA;
+    void* scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (g_noalloc_ptr[dev] == nullptr) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return FLE_ERR_CUDA;
+            g_noalloc_ptr[dev] = p;
+        }
+        scratch = g_noalloc_ptr[dev];
+    }
+    // The plan's scratch need; 0 also for invalid arguments, which
+    // fle_forward then reports.
+    const size_t need = fle_workspace_size(M, K, N, d);
+    if (need > FLE_NOALLOC_SCRATCH_BYTES) return FLE_ERR_WORKSPACE;
+    return fle_forward(x, W, b, M, K, N, d, out, scratch, FLE_NOALLOC_SCRATCH_BYTES, stream);
+}
