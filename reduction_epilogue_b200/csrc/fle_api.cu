@@ -13,6 +13,7 @@
 
 #include "fle.h"
 #include "fle_kernel.cuh"
+#include "fle_kernel_pair.cuh"
 
 namespace {
 
@@ -24,7 +25,33 @@ struct DeviceInfo {
     bool probed = false;
     bool ok = false;
     int sms = 0;
+    int pairs = 0;  // co-resident CTA pairs of the pair kernel (0: pair mode unavailable)
 };
+
+// Co-resident 2-CTA clusters of the pair kernel on the current device.
+int max_active_pairs() {
+    auto kern = fle::fle_gemm_pair_kernel<fle::kPrecTF32>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, fle::PairCfg::kSmemBytes) !=
+        cudaSuccess)
+        return 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(fle::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = fle::PairCfg::kSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
+}
 
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
@@ -44,6 +71,7 @@ int device_info(DeviceInfo* out) {
         d.probed = true;
         d.ok = (major == 10 && minor == 0);
         d.sms = sms;
+        d.pairs = d.ok ? max_active_pairs() : 0;
     }
     if (!d.ok) return FLE_ERR_ARCH;
     if (!g_encode) {
@@ -98,6 +126,7 @@ int check_shape(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d) {
 
 struct Plan {
     bool swap = false;
+    bool pair = false;         // 256x256 tiles on CTA pairs (cta_group::2)
     int bn = 256;
     int prec = fle::kPrecTF32;
     int stages = 0;
@@ -129,25 +158,40 @@ const char* sched_override() {
     return v;
 }
 
-Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int sms) {
+bool pair_disabled() {
+    static bool off = [] {
+        const char* e = std::getenv("FLE_PAIR");
+        return e && e[0] == '0';
+    }();
+    return off;
+}
+
+// sms: SMs of the device; pairs: co-resident CTA pairs of the pair kernel.
+Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int sms, int pairs) {
     Plan pl;
     pl.prec = (d->precision == FLE_PREC_3XTF32) ? fle::kPrec3xTF32 : fle::kPrecTF32;
     pl.swap = (M <= 128) && d->kind != FLE_EPI_AVGPOOL_GELU_SCALE_ROWMAX;
-    if (pl.swap) {
+    pl.pair = !pl.swap && pl.prec == fle::kPrecTF32 && M > 128 && pairs > 0 && !pair_disabled();
+    int tile_m = fle::kBM;
+    if (pl.pair) {
+        tile_m = fle::kPairBM;
+        pl.bn = fle::kPairBN;
+    } else if (pl.swap) {
         pl.bn = M <= 32 ? 32 : (M <= 64 ? 64 : 128);
     } else {
         pl.bn = (pl.prec == fle::kPrec3xTF32) ? 128 : 256;
     }
     const int64_t Ma = pl.swap ? N : M;
     const int64_t Nb = pl.swap ? M : N;
-    pl.tiles_a = static_cast<int>((Ma + fle::kBM - 1) / fle::kBM);
+    pl.tiles_a = static_cast<int>((Ma + tile_m - 1) / tile_m);
     pl.tiles_b = static_cast<int>((Nb + pl.bn - 1) / pl.bn);
     pl.tiles = pl.tiles_a * pl.tiles_b;
     pl.num_kb = static_cast<int>((K + fle::kBK - 1) / fle::kBK);
-    pl.stages = stages_for(pl.bn, pl.prec);
+    pl.stages = pl.pair ? fle::PairCfg::kStages : stages_for(pl.bn, pl.prec);
 
+    // The schedule runs over CTAs, or over CTA pairs in pair mode.
     const int64_t T = pl.tiles;
-    const int64_t G = sms;
+    const int64_t G = pl.pair ? pairs : sms;
     const int64_t iters = T * pl.num_kb;
     // Is a weight tile used by more than one tile of the output?  Then CTAs
     // sharing it must walk K in step to reuse it from L2.
@@ -181,8 +225,12 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
     pl.sk_tiles = static_cast<int>(T - pl.dp_tiles);
     pl.sk_iters = static_cast<int64_t>(pl.sk_tiles) * pl.num_kb;
     if (pl.sk_tiles > 0) {
-        pl.partial_bytes = static_cast<size_t>(2) * pl.sk_grid * fle::kBM * pl.bn * sizeof(float);
-        pl.ws_bytes = pl.partial_bytes + ((static_cast<size_t>(pl.sk_tiles) * 4 + 255) & ~size_t(255));
+        // two fp32 partial tiles of 128 x bn per stream-K CTA, then one
+        // arrival counter per stream-K tile (per CTA of the pair)
+        const int sk_ctas = pl.pair ? 2 * pl.sk_grid : pl.sk_grid;
+        const int counters = pl.pair ? 2 * pl.sk_tiles : pl.sk_tiles;
+        pl.partial_bytes = static_cast<size_t>(2) * sk_ctas * fle::kBM * pl.bn * sizeof(float);
+        pl.ws_bytes = pl.partial_bytes + ((static_cast<size_t>(counters) * 4 + 255) & ~size_t(255));
     }
     return pl;
 }
@@ -204,9 +252,31 @@ cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const KPar
     return cudaGetLastError();
 }
 
+cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const KParams& p, int pairs,
+                             cudaStream_t st) {
+    // max_active_pairs() set the kernel's shared-memory attribute when the
+    // device was probed.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+    cfg.blockDim = dim3(fle::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = fle::PairCfg::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, fle::fle_gemm_pair_kernel<fle::kPrecTF32>, ta, tb, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
 cudaError_t dispatch(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const KParams& p,
                      cudaStream_t st) {
     const bool tf32 = pl.prec == fle::kPrecTF32;
+    if (pl.pair) return launch_gemm_pair(ta, tb, p, pl.grid, st);
     if (!pl.swap) {
         if (tf32 && pl.bn == 256) return launch_gemm<256, fle::kPrecTF32, false>(ta, tb, p, pl.grid, st);
         if (!tf32 && pl.bn == 128) return launch_gemm<128, fle::kPrec3xTF32, false>(ta, tb, p, pl.grid, st);
@@ -255,9 +325,10 @@ bool sync_check_enabled() {
 int plan_to_string(const Plan& pl, char* buf, size_t n) {
     if (!buf || n == 0) return FLE_ERR_NULL;
     std::snprintf(buf, n,
-                  "tile=128x%d swap=%d prec=%s stages=%d tiles=%dx%d kblocks=%d dp_tiles=%d sk_tiles=%d "
+                  "tile=%dx%d pair=%d swap=%d prec=%s stages=%d tiles=%dx%d kblocks=%d dp_tiles=%d sk_tiles=%d "
                   "sk_kblocks=%lld sk_grid=%d grid=%d workspace=%zu",
-                  pl.bn, pl.swap ? 1 : 0, pl.prec == fle::kPrecTF32 ? "tf32" : "3xtf32", pl.stages,
+                  pl.pair ? fle::kPairBM : fle::kBM, pl.bn, pl.pair ? 1 : 0, pl.swap ? 1 : 0,
+                  pl.prec == fle::kPrecTF32 ? "tf32" : "3xtf32", pl.stages,
                   pl.tiles_a, pl.tiles_b, pl.num_kb, pl.dp_tiles, pl.sk_tiles, (long long)pl.sk_iters, pl.sk_grid, pl.grid,
                   pl.ws_bytes);
     return FLE_OK;
@@ -290,7 +361,7 @@ size_t fle_workspace_size(int64_t M, int64_t K, int64_t N, const fle_epilogue_de
     if (M == 0 || N == 0 || K == 0) return 0;
     DeviceInfo di;
     if (device_info(&di) != FLE_OK) return 0;
-    return make_plan(M, K, N, d, di.sms).ws_bytes;
+    return make_plan(M, K, N, d, di.sms, di.pairs).ws_bytes;
 }
 
 int fle_plan_string(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, char* buf, size_t n) {
@@ -301,7 +372,7 @@ int fle_plan_string(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d,
     DeviceInfo di;
     st = device_info(&di);
     if (st != FLE_OK) return st;
-    return plan_to_string(make_plan(M, K, N, d, di.sms), buf, n);
+    return plan_to_string(make_plan(M, K, N, d, di.sms, di.pairs), buf, n);
 }
 
 int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64_t K, int64_t N,
@@ -348,7 +419,7 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
         return cudaGetLastError() == cudaSuccess ? FLE_OK : FLE_ERR_CUDA;
     }
 
-    const Plan pl = make_plan(M, K, N, d, di.sms);
+    const Plan pl = make_plan(M, K, N, d, di.sms, di.pairs);
     if (pl.ws_bytes > 0) {
         if (!workspace || workspace_bytes < pl.ws_bytes) return FLE_ERR_WORKSPACE;
         if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FLE_ERR_ALIGN;
@@ -372,7 +443,7 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
     const float* B = pl.swap ? x : W;
     st = encode_operand(&ta, A, p.Ma, K, fle::kBM);
     if (st != FLE_OK) return st;
-    st = encode_operand(&tb, B, p.Nb, K, pl.bn);
+    st = encode_operand(&tb, B, p.Nb, K, pl.pair ? fle::kPairBN / 2 : pl.bn);
     if (st != FLE_OK) return st;
 
     if (log_enabled()) {
@@ -384,9 +455,10 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
 
     if (pool || pl.sk_tiles > 0) {
         const int threads = 256;
-        const int64_t n = std::max<int64_t>(pool ? M : 0, pl.sk_tiles);
+        const int n_counters = pl.pair ? 2 * pl.sk_tiles : pl.sk_tiles;
+        const int64_t n = std::max<int64_t>(pool ? M : 0, n_counters);
         fle::fle_prep_kernel<<<static_cast<unsigned>((n + threads - 1) / threads), threads, 0, s>>>(
-            pool ? out : nullptr, pool ? M : 0, p.counters, pl.sk_tiles);
+            pool ? out : nullptr, pool ? M : 0, p.counters, n_counters);
         if (cudaGetLastError() != cudaSuccess) return FLE_ERR_CUDA;
     }
     if (dispatch(pl, ta, tb, p, s) != cudaSuccess) return FLE_ERR_CUDA;
@@ -404,7 +476,7 @@ int fle_plan_units(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, 
     *n_units = 0;
     if (grid) *grid = 0;
     if (M == 0 || N == 0 || K == 0) return FLE_OK;
-    const Plan pl = make_plan(M, K, N, d, num_sms);
+    const Plan pl = make_plan(M, K, N, d, num_sms, num_sms / 2);
     if (grid) *grid = pl.grid;
     if (cta >= pl.grid) return FLE_OK;
     KParams p{};

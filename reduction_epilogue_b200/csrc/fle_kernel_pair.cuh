@@ -1,0 +1,279 @@
+// fle_kernel_pair.cuh -- the fused Linear + epilogue kernel on CTA pairs.
+//
+// Two CTAs of a cluster, on two SMs, compute one 256 x 256 output tile with
+// tcgen05.mma.cta_group::2: each CTA loads its own 128 rows of A (x) and its
+// own 128 rows of B (W) into its shared memory, and the pair's MMA reads A and
+// B from both.  Per SM this halves the B operand traffic through shared memory
+// compared with a 128 x 256 single-CTA tile, at the same MMA work per SM.
+// The accumulator rows are split across the two SMs' TMEM (rows 0-127 in the
+// even CTA, 128-255 in the odd one), so each CTA runs the epilogue of its own
+// 128 rows.
+//
+// Roles are those of fle_gemm_kernel.  Only the even ("leader") CTA's MMA
+// thread issues MMAs; both CTAs' producers load, and their copies are counted
+// on the leader's full barrier; the leader's commits are multicast to both
+// CTAs' empty and accumulator-full barriers; both CTAs' epilogues release the
+// leader's accumulator-empty barrier.  No load uses cluster multicast.
+#pragma once
+
+#include "fle_kernel.cuh"
+
+namespace fle {
+
+constexpr int kPairBN = 256;                      // pair tile N (B rows)
+constexpr int kPairBM = 256;                      // pair tile M (A rows)
+
+struct PairCfg {
+    static constexpr int kABytes = kBM * kBK * 4;          // this CTA's 128 A rows
+    static constexpr int kBBytes = (kPairBN / 2) * kBK * 4;  // this CTA's 128 B rows
+    static constexpr int kLoadBytes = kABytes + kBBytes;
+    static constexpr int kStages = kSmemStageBudget / kLoadBytes > 8 ? 8 : kSmemStageBudget / kLoadBytes;
+    static constexpr int kTmemCols = 512;                    // 2 accumulator buffers x 256 columns
+    // full, empty per stage; accf, acce per buffer; drain; exit
+    static constexpr int kNumBars = 2 * kStages + 4 + 2;
+    static constexpr int kSmemBytes = 1024 + kStages * kLoadBytes + kNumBars * 8 + 32;
+};
+
+template <int PREC>
+__global__ void __launch_bounds__(kThreads, 1)
+fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const KParams p) {
+    static_assert(PREC == kPrecTF32, "CTA-pair kernel: single-pass TF32");
+    using C = PairCfg;
+    constexpr int S = C::kStages;
+    constexpr uint32_t kIdesc = idesc_tf32(kPairBM, kPairBN);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kLoadBytes);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+    auto bar_full = [&](int s) { return smem_u32(bars + s); };
+    auto bar_empty = [&](int s) { return smem_u32(bars + S + s); };
+    auto bar_accf = [&](int b) { return smem_u32(bars + 2 * S + b); };
+    auto bar_acce = [&](int b) { return smem_u32(bars + 2 * S + 2 + b); };
+    const uint32_t bar_drain = smem_u32(bars + 2 * S + 4);
+    const uint32_t bar_exit = smem_u32(bars + 2 * S + 5);
+    auto sA = [&](int s) { return sbase + s * C::kLoadBytes; };
+    auto sB = [&](int s) { return sbase + s * C::kLoadBytes + C::kABytes; };
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();  // 0: leader, 1: peer
+    const int pair = blockIdx.x >> 1;
+    const int num_pairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(bar_full(s), 1);
+            mbar_init(bar_empty(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_accf(b), 1);
+            mbar_init(bar_acce(b), 8);  // 4 epilogue warps in each CTA of the pair
+        }
+        mbar_init(bar_drain, 1);
+        mbar_init(bar_exit, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(tmem_slot), C::kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before_sync();
+    cluster_sync_all();  // both CTAs' barriers exist before either signals the other
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer (both CTAs)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            long long fills = 0;
+            bool ok = true;
+            Sched sc;
+            sc.init(p, pair, num_pairs);
+            Unit u;
+            while (ok && sc.next(p, u)) {
+                for (int kb = u.kb0; kb < u.kb1; ++kb) {
+                    if (!mbar_wait_bounded(bar_empty(stage), phase ^ 1u, abort_flag, p.timeout_ns,
+                                           kWhereProdEmpty)) {
+                        ok = false;
+                        break;
+                    }
+                    // The leader expects both CTAs' bytes on its own full barrier.
+                    if (rank == 0) mbar_arrive_expect_tx(bar_full(stage), 2 * C::kLoadBytes);
+                    const uint32_t leader_full = mapa_shared(bar_full(stage), 0);
+                    tma_load_2d_pair(sA(stage), &tmA, leader_full, kb * kBK, u.ta * kPairBM + rank * kBM);
+                    tma_load_2d_pair(sB(stage), &tmB, leader_full, kb * kBK, u.tb * kPairBN + rank * (kPairBN / 2));
+                    ++fills;
+                    if (++stage == S) { stage = 0; phase ^= 1u; }
+                }
+            }
+            // This CTA's copies land before its stages are released by the
+            // leader's MMA commit; wait for that on the last stages filled.
+            for (long long f = (fills > S ? fills - S : 0); f < fills; ++f) {
+                const int s = static_cast<int>(f % S);
+                const uint32_t ph = static_cast<uint32_t>((f / S) & 1);
+                volatile int never = 0;
+                mbar_wait_bounded(bar_empty(s), ph, &never, p.timeout_ns, kWhereProdDrain);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (leader only)
+        if (lane == 0 && rank == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int buf = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            Sched sc;
+            sc.init(p, pair, num_pairs);
+            Unit u;
+            while (ok && sc.next(p, u)) {
+                if (!mbar_wait_bounded(bar_acce(buf), acc_phase ^ 1u, abort_flag, p.timeout_ns,
+                                       kWhereMmaAccEmpty)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kPairBN);
+                for (int kb = u.kb0; kb < u.kb1; ++kb) {
+                    if (!mbar_wait_bounded(bar_full(stage), phase, abort_flag, p.timeout_ns, kWhereMmaFull)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint64_t a_desc = smem_desc_sw128(sA(stage));
+                    const uint64_t b_desc = smem_desc_sw128(sB(stage));
+#pragma unroll
+                    for (int k = 0; k < kBK / kUmmaK; ++k) {
+                        const uint64_t koff = static_cast<uint64_t>(k * 2);
+                        mma_tf32_pair(d_tmem, a_desc + koff, b_desc + koff, kIdesc, (kb > u.kb0 || k > 0) ? 1u : 0u);
+                    }
+                    mma_commit_pair_multicast(bar_empty(stage), 0x3);
+                    if (++stage == S) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                mma_commit_pair_multicast(bar_accf(buf), 0x3);
+                buf ^= 1;
+                if (buf == 0) acc_phase ^= 1u;
+            }
+            mma_commit_pair(bar_drain);
+            volatile int never = 0;
+            mbar_wait_bounded(bar_drain, 0, &never, p.timeout_ns, kWhereDrain);
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int q = warp - 4;
+        const int r = q * 32 + lane;
+        int buf = 0;
+        uint32_t acc_phase = 0;
+        Sched sc;
+        sc.init(p, pair, num_pairs);
+        Unit u;
+        while (sc.next(p, u)) {
+            int got = 0;
+            if (lane == 0)
+                got = mbar_wait_bounded(bar_accf(buf), acc_phase, abort_flag, p.timeout_ns, kWhereEpiAccFull);
+            got = __shfl_sync(0xffffffffu, got, 0);
+            if (!got) break;
+            tc_fence_after_sync();
+            const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * kPairBN);
+            const int64_t cols_left = p.N - static_cast<int64_t>(u.tb) * kPairBN;
+            const int nchunks = static_cast<int>(cols_left >= kPairBN ? kPairBN / 32 : (cols_left + 31) / 32);
+            // This CTA's 128 rows of the pair tile, as a 128-row tile index.
+            Unit uh = u;
+            uh.ta = 2 * u.ta + static_cast<int>(rank);
+            auto release_acc = [&]() {
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(bar_acce(buf), 0));
+                buf ^= 1;
+                if (buf == 0) acc_phase ^= 1u;
+            };
+
+            if (!u.partial) {
+                float best = -INFINITY;
+#pragma unroll 1
+                for (int c = 0; c < nchunks; ++c) {
+                    float v[32];
+                    tmem_ld32_wait(t_acc + c * 32, v);
+                    epi_chunk<false, kPairBN>(p, uh, r, c, v, best);
+                }
+                epi_finish<false>(p, uh, r, best);
+                release_acc();
+            } else {
+                float* mine = p.ws + (static_cast<size_t>(2 * blockIdx.x + u.slot) * kBM + r) * kPairBN;
+#pragma unroll 1
+                for (int c = 0; c < nchunks; ++c) {
+                    float v[32];
+                    tmem_ld32_wait(t_acc + c * 32, v);
+                    float4* d4 = reinterpret_cast<float4*>(mine + c * 32);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        __stcg(d4 + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+                }
+                release_acc();
+                const int64_t tsk = u.sk_tile;
+                const int first = sk_cta_of(tsk * p.num_kb, p.sk_iters, p.sk_grid);
+                const int last = sk_cta_of((tsk + 1) * p.num_kb - 1, p.sk_iters, p.sk_grid);
+                unsigned* counter = p.counters + 2 * tsk + rank;
+                __threadfence();
+                epilogue_bar_sync();
+                if (threadIdx.x == 128) {
+                    const unsigned prev = atomicAdd(counter, 1u);
+                    *last_flag = (prev == static_cast<unsigned>(last - first)) ? 1 : 0;
+                }
+                epilogue_bar_sync();
+                if (*last_flag) {
+                    __threadfence();
+                    float best = -INFINITY;
+                    for (int c = 0; c < nchunks; ++c) {
+                        float v[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+                        for (int cc = first; cc <= last; ++cc) {
+                            const int sl = sk_slot_of(cc, tsk, p.sk_iters, p.sk_grid, p.num_kb);
+                            const float4* s4 = reinterpret_cast<const float4*>(
+                                p.ws + (static_cast<size_t>(2 * (2 * cc + rank) + sl) * kBM + r) * kPairBN + c * 32);
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const float4 t = __ldcg(s4 + j);
+                                v[4 * j] += t.x; v[4 * j + 1] += t.y; v[4 * j + 2] += t.z; v[4 * j + 3] += t.w;
+                            }
+                        }
+                        epi_chunk<false, kPairBN>(p, uh, r, c, v, best);
+                    }
+                    epi_finish<false>(p, uh, r, best);
+                    if (threadIdx.x == 128) *counter = 0u;
+                }
+            }
+        }
+    }
+
+    // Neither CTA may release TMEM or exit while the other can still signal
+    // its barriers or (leader) write its TMEM: a bounded two-way handshake.
+    tc_fence_before_sync();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        mbar_arrive_cluster(mapa_shared(bar_exit, rank ^ 1u));
+        volatile int never = 0;
+        mbar_wait_bounded(bar_exit, 0, &never, p.timeout_ns, kWhereDrain);
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    }
+}
+
+}  // namespace fle

@@ -70,8 +70,9 @@ def test_schedule_covers_every_kblock_once(M, K, N, problem, precision, sms):
     tas = {e[3][0] for v in cover.values() for e in v}
     tbs = {e[3][1] for v in cover.values() for e in v}
     assert len(tas) * len(tbs) == len(tiles)
-    # the tiles span exactly the operand rows (A side holds M or N)
-    a_rows = {math.ceil(M / 128), math.ceil(N / 128)}
+    # the tiles span exactly the operand rows (A side holds M or N, in tiles
+    # of 128 rows, or 256 rows on CTA pairs)
+    a_rows = {math.ceil(M / 128), math.ceil(N / 128), math.ceil(M / 256)}
     assert len(tas) in a_rows
 
     for t, units in cover.items():
@@ -99,18 +100,22 @@ def test_schedule_covers_every_kblock_once(M, K, N, problem, precision, sms):
 
 
 def test_headline_shape_splits_only_the_last_wave():
-    # 2048x8192x8192 with 128x256 tiles: 512 tiles on 148 SMs is 3.46 waves.
-    # Three waves run whole tiles; the 68 tiles of the last wave are split in
-    # two k-aligned halves on 136 CTAs, so the SMs finish within half a tile.
+    # 2048x8192x8192 in TF32 runs 256x256 tiles on CTA pairs: 256 tiles on the
+    # 74 pairs of 148 SMs is 3.46 waves.  Three waves run whole tiles; the 34
+    # tiles of the last wave are split in two k-aligned halves on 68 pairs, so
+    # the pairs finish within half a tile.
     desc = fle.desc_for("scale_hardtanh_gelu", "tf32")
     grid, per_cta = collect(2048, 8192, 8192, desc, 148)
-    assert grid == 148
+    assert grid == 74
     load = [sum(int(r[4]) - int(r[3]) for r in rows) for rows in per_cta]
-    assert sum(load) == 512 * 256
+    assert sum(load) == 256 * 256
     assert max(load) - min(load) == 128
     halves = [r for rows in per_cta for r in rows if r[5]]
-    assert len(halves) == 136
+    assert len(halves) == 68
     assert {(int(r[3]), int(r[4])) for r in halves} == {(0, 128), (128, 256)}
+    # 3xTF32 keeps single-CTA 128x128 tiles: 16 x 64 = 1024 tiles
+    grid3, per3 = collect(2048, 8192, 8192, fle.desc_for("scale_hardtanh_gelu", "3xtf32"), 148)
+    assert grid3 == 148 and sum(len(r) for r in per3) == 1024
 
 
 def test_weight_streamed_once_shapes_use_every_sm():
