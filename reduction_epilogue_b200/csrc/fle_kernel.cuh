@@ -18,11 +18,12 @@
 // dimension sits on the 128-row side of the MMA; either way both operands are
 // K-major, as nn.Linear stores them.
 //
-// Warp roles (256 threads):
+// Warp roles (384 threads):
 //   warp 0, lane 0   TMA producer: fills a ring of shared-memory stages.
 //   warp 1           allocates TMEM; lane 0 issues the tcgen05.mma chain.
 //   warps 2-3        3xTF32 only: split each landed stage into TF32 hi/lo parts.
-//   warps 4-7        epilogue: TMEM -> registers -> bias + epilogue -> global.
+//   warps 4-11       epilogue: TMEM -> registers -> bias + epilogue -> global;
+//                    two warps per TMEM lane quadrant, each with half the columns.
 // The accumulator is double-buffered in TMEM, so the epilogue of one tile
 // overlaps the main loop of the next.
 #pragma once
@@ -38,8 +39,8 @@ namespace fle {
 constexpr int kBM = 128;           // MMA M: rows of operand A per tile
 constexpr int kBK = 32;            // fp32 per k-block = one 128-byte swizzled row
 constexpr int kUmmaK = 8;          // K of one tcgen05.mma kind::tf32
-constexpr int kThreads = 256;
-constexpr int kSmemStageBudget = 196608;  // bytes of shared memory for stages
+constexpr int kThreads = 384;
+constexpr int kSmemStageBudget = 229376;  // bytes of shared memory for stages (224 KB)
 
 enum : int { kEpiHardtanhGelu = 0, kEpiSwish = 1, kEpiPoolMax = 2, kEpiNone = 3 };
 enum : int { kPrec3xTF32 = 0, kPrecTF32 = 1 };
@@ -293,9 +294,9 @@ __device__ __forceinline__ void epi_finish(const KParams& p, const Unit& u, int 
     }
 }
 
-// Barrier among the four epilogue warps only (named barrier 1, 128 threads).
+// Barrier among the eight epilogue warps only (named barrier 1, 256 threads).
 __device__ __forceinline__ void epilogue_bar_sync() {
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    asm volatile("bar.sync 1, 256;" ::: "memory");
 }
 
 // ----------------------------------------------------------------------------
@@ -340,7 +341,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_accf(b), 1);
-            mbar_init(bar_acce(b), 4);
+            mbar_init(bar_acce(b), 8);  // one arrival per epilogue warp
         }
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
@@ -493,8 +494,16 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int q = warp - 4;       // TMEM lane quadrant of this warp
+        // Eight warps.  Warp w reads TMEM lane quadrant w % 4 (tile rows
+        // 32*(w%4) .. +31; a warp may only touch its own quadrant) and one
+        // half of the tile's 32-column chunks, so each SM sub-partition runs
+        // two independent epilogue warps.
+        const int q = warp & 3;
+        const int half = (warp - 4) >> 2;
         const int r = q * 32 + lane;  // tile row = TMEM lane of this thread
+        constexpr int kChunks = BN / 32;
+        constexpr int kHalf = (kChunks + 1) / 2;  // chunks per half
+        const int c_lo = half * kHalf;
         int buf = 0;
         uint32_t acc_phase = 0;
         // 3xTF32 accumulates each kChunkKb-deep slice of K in a fresh TMEM
@@ -502,15 +511,17 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         // round-to-nearest: the tensor core's own accumulation rounds toward
         // zero, whose bias would otherwise grow with the length of K.
         constexpr bool kRegAcc = (PREC == kPrec3xTF32);
-        float accr[kRegAcc ? BN : 1];
+        float accr[kRegAcc ? kHalf * 32 : 1];
         Sched sc;
         sc.init(p, blockIdx.x, gridDim.x);
         Unit u;
         bool ok = true;
         while (ok && sc.next(p, u)) {
-            // 32-column chunks of this tile that hold any output (warp-uniform)
+            // 32-column chunks of this tile that hold any output, and this
+            // warp's share [c_lo, c_lo + mine) of them (warp-uniform)
             const int64_t cols_left = (SWAP ? p.M : p.N) - static_cast<int64_t>(u.tb) * BN;
-            const int nchunks = static_cast<int>(cols_left >= BN ? BN / 32 : (cols_left + 31) / 32);
+            const int nchunks = static_cast<int>(cols_left >= BN ? kChunks : (cols_left + 31) / 32);
+            const int mine = nchunks - c_lo < 0 ? 0 : (nchunks - c_lo > kHalf ? kHalf : nchunks - c_lo);
 
             auto wait_acc = [&]() -> bool {
                 int got = 0;
@@ -534,17 +545,17 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             uint32_t t_acc = 0;
             if constexpr (kRegAcc) {
 #pragma unroll
-                for (int j = 0; j < (kRegAcc ? BN : 1); ++j) accr[j] = 0.0f;
+                for (int j = 0; j < (kRegAcc ? kHalf * 32 : 1); ++j) accr[j] = 0.0f;
                 for (int kc = u.kb0; kc < u.kb1; kc += kChunkKb) {
                     if (!wait_acc()) { ok = false; break; }
                     const uint32_t tr = t_row();
 #pragma unroll
-                    for (int c = 0; c < BN / 32; ++c) {
-                        if (c >= nchunks) break;
+                    for (int lc = 0; lc < kHalf; ++lc) {
+                        if (lc >= mine) break;
                         float v[32];
-                        tmem_ld32_wait(tr + c * 32, v);
+                        tmem_ld32_wait(tr + (c_lo + lc) * 32, v);
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) accr[c * 32 + j] += v[j];
+                        for (int j = 0; j < 32; ++j) accr[lc * 32 + j] += v[j];
                     }
                     release_acc();
                 }
@@ -553,55 +564,56 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 if (!wait_acc()) break;
                 t_acc = t_row();
             }
-            // The 32 accumulator values of chunk c of this unit, in registers
-            // (3xTF32) or in TMEM (TF32).  Called with compile-time c when the
-            // values are registers.
-#define FLE_LOAD_ACC(c, v)                                                        \
-    do {                                                                          \
-        if constexpr (kRegAcc) {                                                  \
-            _Pragma("unroll") for (int j_ = 0; j_ < 32; ++j_) v[j_] = accr[(c) * 32 + j_]; \
-        } else {                                                                  \
-            tmem_ld32_wait(t_acc + (c) * 32, v);                                  \
-        }                                                                         \
+            // The 32 accumulator values of this warp's local chunk lc, in
+            // registers (3xTF32, with compile-time lc) or in TMEM (TF32).
+#define FLE_LOAD_ACC(lc, v)                                                                    \
+    do {                                                                                       \
+        if constexpr (kRegAcc) {                                                               \
+            _Pragma("unroll") for (int j_ = 0; j_ < 32; ++j_) v[j_] = accr[(lc) * 32 + j_];    \
+        } else {                                                                               \
+            tmem_ld32_wait(t_acc + (c_lo + (lc)) * 32, v);                                     \
+        }                                                                                      \
     } while (0)
 
             if (!u.partial) {
                 float best = -INFINITY;
-#define FLE_EPI_BODY(c)                          \
-    {                                            \
-        float v[32];                             \
-        FLE_LOAD_ACC(c, v);                      \
-        epi_chunk<SWAP, BN>(p, u, r, c, v, best); \
+#define FLE_EPI_BODY(lc)                                     \
+    {                                                        \
+        float v[32];                                         \
+        FLE_LOAD_ACC(lc, v);                                 \
+        epi_chunk<SWAP, BN>(p, u, r, c_lo + (lc), v, best);  \
     }
                 if constexpr (kRegAcc) {
 #pragma unroll
-                    for (int c = 0; c < BN / 32; ++c)
-                        if (c < nchunks) FLE_EPI_BODY(c)
+                    for (int lc = 0; lc < kHalf; ++lc)
+                        if (lc < mine) FLE_EPI_BODY(lc)
                 } else {
 #pragma unroll 1
-                    for (int c = 0; c < nchunks; ++c) FLE_EPI_BODY(c)
+                    for (int lc = 0; lc < mine; ++lc) FLE_EPI_BODY(lc)
                 }
 #undef FLE_EPI_BODY
                 epi_finish<SWAP>(p, u, r, best);
                 if constexpr (!kRegAcc) release_acc();
             } else {
-                // Park this CTA's fp32 partial tile in its workspace slot.
-                float* mine = p.ws + (static_cast<size_t>(2 * blockIdx.x + u.slot) * kBM + r) * BN;
-#define FLE_PARK_BODY(c)                                                                            \
-    {                                                                                               \
-        float v[32];                                                                                \
-        FLE_LOAD_ACC(c, v);                                                                         \
-        float4* d4 = reinterpret_cast<float4*>(mine + (c) * 32);                                    \
-        _Pragma("unroll") for (int j = 0; j < 8; ++j)                                               \
-            __stcg(d4 + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));        \
+                // Park this CTA's fp32 partial tile in its workspace slot,
+                // column-major inside the tile (element (row, col) at
+                // col * 128 + row) so that a warp's lanes write 32 consecutive
+                // floats.
+                float* slot = p.ws + static_cast<size_t>(2 * blockIdx.x + u.slot) * kBM * BN;
+#define FLE_PARK_BODY(lc)                                                                 \
+    {                                                                                     \
+        float v[32];                                                                      \
+        FLE_LOAD_ACC(lc, v);                                                              \
+        float* d = slot + static_cast<size_t>((c_lo + (lc)) * 32) * kBM + r;              \
+        _Pragma("unroll") for (int j = 0; j < 32; ++j) __stcg(d + j * kBM, v[j]);         \
     }
                 if constexpr (kRegAcc) {
 #pragma unroll
-                    for (int c = 0; c < BN / 32; ++c)
-                        if (c < nchunks) FLE_PARK_BODY(c)
+                    for (int lc = 0; lc < kHalf; ++lc)
+                        if (lc < mine) FLE_PARK_BODY(lc)
                 } else {
 #pragma unroll 1
-                    for (int c = 0; c < nchunks; ++c) FLE_PARK_BODY(c)
+                    for (int lc = 0; lc < mine; ++lc) FLE_PARK_BODY(lc)
                 }
 #undef FLE_PARK_BODY
                 if constexpr (!kRegAcc) release_acc();
@@ -620,19 +632,21 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     // order (= k order), then run the epilogue on the sum.
                     __threadfence();
                     float best = -INFINITY;
-                    for (int c = 0; c < nchunks; ++c) {
+#pragma unroll 1
+                    for (int lc = 0; lc < mine; ++lc) {
+                        const int c = c_lo + lc;
                         float v[32];
 #pragma unroll
                         for (int j = 0; j < 32; ++j) v[j] = 0.0f;
                         for (int cc = first; cc <= last; ++cc) {
                             const int sl = sk_slot_of(cc, tsk, p.sk_iters, p.sk_grid, p.num_kb);
-                            const float4* s4 = reinterpret_cast<const float4*>(
-                                p.ws + (static_cast<size_t>(2 * cc + sl) * kBM + r) * BN + c * 32);
+                            const float* src = p.ws + static_cast<size_t>(2 * cc + sl) * kBM * BN +
+                                               static_cast<size_t>(c * 32) * kBM + r;
+                            float t[32];
 #pragma unroll
-                            for (int j = 0; j < 8; ++j) {
-                                const float4 t = __ldcg(s4 + j);
-                                v[4 * j] += t.x; v[4 * j + 1] += t.y; v[4 * j + 2] += t.z; v[4 * j + 3] += t.w;
-                            }
+                            for (int j = 0; j < 32; ++j) t[j] = __ldcg(src + j * kBM);
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] += t[j];
                         }
                         epi_chunk<SWAP, BN>(p, u, r, c, v, best);
                     }

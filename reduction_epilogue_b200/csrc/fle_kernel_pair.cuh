@@ -27,7 +27,7 @@ struct PairCfg {
     static constexpr int kABytes = kBM * kBK * 4;          // this CTA's 128 A rows
     static constexpr int kBBytes = (kPairBN / 2) * kBK * 4;  // this CTA's 128 B rows
     static constexpr int kLoadBytes = kABytes + kBBytes;
-    static constexpr int kStages = kSmemStageBudget / kLoadBytes > 8 ? 8 : kSmemStageBudget / kLoadBytes;
+    static constexpr int kStages = 7;  // 224 KB of stages; the tile needs no other shared memory
     static constexpr int kTmemCols = 512;                    // 2 accumulator buffers x 256 columns
     // full, empty per stage; accf, acce per buffer; drain; exit
     static constexpr int kNumBars = 2 * kStages + 4 + 2;
@@ -73,7 +73,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_accf(b), 1);
-            mbar_init(bar_acce(b), 8);  // 4 epilogue warps in each CTA of the pair
+            mbar_init(bar_acce(b), 16);  // 8 epilogue warps in each CTA of the pair
         }
         mbar_init(bar_drain, 1);
         mbar_init(bar_exit, 1);
@@ -173,8 +173,12 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         __syncwarp();
     } else if (warp >= 4) {
         // ------------------------------------------------------------ epilogue (both CTAs)
-        const int q = warp - 4;
+        // Eight warps: lane quadrant warp % 4, half of the columns each.
+        const int q = warp & 3;
+        const int half = (warp - 4) >> 2;
         const int r = q * 32 + lane;
+        constexpr int kHalf = kPairBN / 32 / 2;  // chunks per half
+        const int c_lo = half * kHalf;
         int buf = 0;
         uint32_t acc_phase = 0;
         Sched sc;
@@ -190,6 +194,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * kPairBN);
             const int64_t cols_left = p.N - static_cast<int64_t>(u.tb) * kPairBN;
             const int nchunks = static_cast<int>(cols_left >= kPairBN ? kPairBN / 32 : (cols_left + 31) / 32);
+            const int mine = nchunks - c_lo < 0 ? 0 : (nchunks - c_lo > kHalf ? kHalf : nchunks - c_lo);
             // This CTA's 128 rows of the pair tile, as a 128-row tile index.
             Unit uh = u;
             uh.ta = 2 * u.ta + static_cast<int>(rank);
@@ -204,23 +209,23 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             if (!u.partial) {
                 float best = -INFINITY;
 #pragma unroll 1
-                for (int c = 0; c < nchunks; ++c) {
+                for (int lc = 0; lc < mine; ++lc) {
                     float v[32];
-                    tmem_ld32_wait(t_acc + c * 32, v);
-                    epi_chunk<false, kPairBN>(p, uh, r, c, v, best);
+                    tmem_ld32_wait(t_acc + (c_lo + lc) * 32, v);
+                    epi_chunk<false, kPairBN>(p, uh, r, c_lo + lc, v, best);
                 }
                 epi_finish<false>(p, uh, r, best);
                 release_acc();
             } else {
-                float* mine = p.ws + (static_cast<size_t>(2 * blockIdx.x + u.slot) * kBM + r) * kPairBN;
+                // column-major partial tile: element (row, col) at col * 128 + row
+                float* slot = p.ws + static_cast<size_t>(2 * blockIdx.x + u.slot) * kBM * kPairBN;
 #pragma unroll 1
-                for (int c = 0; c < nchunks; ++c) {
+                for (int lc = 0; lc < mine; ++lc) {
                     float v[32];
-                    tmem_ld32_wait(t_acc + c * 32, v);
-                    float4* d4 = reinterpret_cast<float4*>(mine + c * 32);
+                    tmem_ld32_wait(t_acc + (c_lo + lc) * 32, v);
+                    float* d = slot + static_cast<size_t>((c_lo + lc) * 32) * kBM + r;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        __stcg(d4 + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+                    for (int j = 0; j < 32; ++j) __stcg(d + j * kBM, v[j]);
                 }
                 release_acc();
                 const int64_t tsk = u.sk_tile;
@@ -237,19 +242,21 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 if (*last_flag) {
                     __threadfence();
                     float best = -INFINITY;
-                    for (int c = 0; c < nchunks; ++c) {
+#pragma unroll 1
+                    for (int lc = 0; lc < mine; ++lc) {
+                        const int c = c_lo + lc;
                         float v[32];
 #pragma unroll
                         for (int j = 0; j < 32; ++j) v[j] = 0.0f;
                         for (int cc = first; cc <= last; ++cc) {
                             const int sl = sk_slot_of(cc, tsk, p.sk_iters, p.sk_grid, p.num_kb);
-                            const float4* s4 = reinterpret_cast<const float4*>(
-                                p.ws + (static_cast<size_t>(2 * (2 * cc + rank) + sl) * kBM + r) * kPairBN + c * 32);
+                            const float* src = p.ws + static_cast<size_t>(2 * (2 * cc + rank) + sl) * kBM * kPairBN +
+                                               static_cast<size_t>(c * 32) * kBM + r;
+                            float t[32];
 #pragma unroll
-                            for (int j = 0; j < 8; ++j) {
-                                const float4 t = __ldcg(s4 + j);
-                                v[4 * j] += t.x; v[4 * j + 1] += t.y; v[4 * j + 2] += t.z; v[4 * j + 3] += t.w;
-                            }
+                            for (int j = 0; j < 32; ++j) t[j] = __ldcg(src + j * kBM);
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] += t[j];
                         }
                         epi_chunk<false, kPairBN>(p, uh, r, c, v, best);
                     }
