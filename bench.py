@@ -41,6 +41,13 @@ CONFIGS = {
     "sweep_m256_k8192_n8192_hardtanh_gelu": (256, 8192, 8192, "scale_hardtanh_gelu"),
     "sweep_m1024_k8192_n8192_hardtanh_gelu": (1024, 8192, 8192, "scale_hardtanh_gelu"),
     "sweep_m4096_k8192_n8192_hardtanh_gelu": (4096, 8192, 8192, "scale_hardtanh_gelu"),
+    # epilogue (c) by pooled weights: pool W and b every call, or reuse them
+    "poolfold_per_call_1024x8192x8192_pool16_gelu_rowmax": (1024, 8192, 8192, "avgpool_gelu_scale_rowmax"),
+    "poolfold_cached_1024x8192x8192_pool16_gelu_rowmax": (1024, 8192, 8192, "avgpool_gelu_scale_rowmax"),
+}
+VARIANT = {
+    "poolfold_per_call_1024x8192x8192_pool16_gelu_rowmax": "poolfold",
+    "poolfold_cached_1024x8192x8192_pool16_gelu_rowmax": "poolfold_cached",
 }
 DEFAULT_CONFIG = "linear2048x8192x8192_hardtanh_gelu"
 
@@ -89,9 +96,19 @@ def profiled_traffic(workload: str, precision: str):
         return None
 
 
-def algorithmic(M, K, N, problem):
-    flops = 2.0 * M * N * K
+def algorithmic(M, K, N, problem, variant=None):
+    """(flops, bytes, output elements) one call must do.  The pooled-weight
+    variants do the GEMM at N/16 columns; per call they also read W once and
+    write and read the pooled weights."""
     out_elems = M if problem == "avgpool_gelu_scale_rowmax" else M * N
+    if variant in ("poolfold", "poolfold_cached"):
+        P = N // 16
+        flops = 2.0 * M * P * K
+        nbytes = 4.0 * (M * K + P * K + P + out_elems)
+        if variant == "poolfold":
+            nbytes += 4.0 * (N * K + N + P * K + P)
+        return flops, nbytes, out_elems
+    flops = 2.0 * M * N * K
     nbytes = 4.0 * (M * K + N * K + N + out_elems)
     return flops, nbytes, out_elems
 
@@ -227,21 +244,43 @@ def run_fle(args, name, dist_ctx):
 
     rank, world, dev = dist_ctx
     M, K, N, problem = CONFIGS[name]
-    flops, nbytes, out_elems = algorithmic(M, K, N, problem)
+    variant = VARIANT.get(name)
+    flops, nbytes, out_elems = algorithmic(M, K, N, problem, variant)
     desc = fle.desc_for(problem, args.precision)
     x, W, b = synth.linear_inputs(M, K, N, seed=rank, device=dev)
     out = torch.empty((M,) if problem == "avgpool_gelu_scale_rowmax" else (M, N), device=dev)
-    ws_bytes = fle.workspace_size(M, K, N, desc)
-    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-    launches_per_step = 2 if problem == "avgpool_gelu_scale_rowmax" else 1
+    plan_shape = (M, K, N, desc)
+    if variant == "poolfold":
+        ws_bytes = fle.workspace_size_pooled(M, K, N, desc)
+        ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+        fdesc = fle.desc_for(problem, args.precision, pool_k=1)
+        plan_shape = (M, K, N // 16, fdesc)
+
+        def step():
+            fle.forward_pooled(x, W, b, out, desc, workspace=ws, workspace_bytes=ws_bytes, stream=stream)
+    elif variant == "poolfold_cached":
+        Wp, bp = fle.pool_weights(W, b, 16, stream=stream)
+        fdesc = fle.desc_for(problem, args.precision, pool_k=1)
+        ws_bytes = fle.workspace_size(M, K, N // 16, fdesc)
+        ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+        plan_shape = (M, K, N // 16, fdesc)
+
+        def step():
+            fle.forward(x, Wp, bp, out, fdesc, workspace=ws, workspace_bytes=ws_bytes, stream=stream)
+    else:
+        ws_bytes = fle.workspace_size(M, K, N, desc)
+        ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+
+        def step():
+            fle.forward(x, W, b, out, desc, workspace=ws, workspace_bytes=ws_bytes, stream=stream)
+    launches_per_step = (2 if problem == "avgpool_gelu_scale_rowmax" else 1) + (1 if variant == "poolfold" else 0)
 
     input_bytes = 4 * (M * K + N * K + N)
+    if variant == "poolfold_cached":
+        input_bytes = 4 * (M * K + (N // 16) * K + N // 16)
     flush = input_bytes <= 2 * L2_BYTES
     scrub = torch.empty(2 * L2_BYTES // 4, device=dev) if flush else None
-
-    def step():
-        fle.forward(x, W, b, out, desc, workspace=ws, workspace_bytes=ws_bytes, stream=stream)
 
     for _ in range(args.warmup):
         if flush:
@@ -286,8 +325,16 @@ def run_fle(args, name, dist_ctx):
         bh = b.cpu().pin_memory()
         outh = torch.empty(out.shape, dtype=torch.float32).pin_memory()
         e2e_steps = max(1, min(args.steps, args.e2e_steps))
+        copy_w = variant != "poolfold_cached"  # cached pooled weights stay on the device
+
+        def h2d():
+            x.copy_(xh, non_blocking=True)
+            if copy_w:
+                W.copy_(Wh, non_blocking=True)
+                b.copy_(bh, non_blocking=True)
+
         for _ in range(2):
-            x.copy_(xh, non_blocking=True); W.copy_(Wh, non_blocking=True); b.copy_(bh, non_blocking=True)
+            h2d()
             step()
             outh.copy_(out, non_blocking=True)
         if world > 1:
@@ -297,7 +344,7 @@ def run_fle(args, name, dist_ctx):
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(e2e_steps):
-            x.copy_(xh, non_blocking=True); W.copy_(Wh, non_blocking=True); b.copy_(bh, non_blocking=True)
+            h2d()
             step()
             outh.copy_(out, non_blocking=True)
         e1.record(stream)
@@ -306,7 +353,8 @@ def run_fle(args, name, dist_ctx):
         if world > 1:
             torch.distributed.all_reduce(e_ms, op=torch.distributed.ReduceOp.MAX)
         e2e = {"value": flops * world * e2e_steps / (float(e_ms.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": input_bytes, "d2h_bytes_per_step": 4 * out_elems, "steps": e2e_steps}
+               "h2d_bytes_per_step": (4 * (M * K + N * K + N) if copy_w else 4 * M * K),
+               "d2h_bytes_per_step": 4 * out_elems, "steps": e2e_steps}
 
     # roofline of the dominant (only) kernel
     peaks, peak_src = load_peaks()
@@ -338,7 +386,7 @@ def run_fle(args, name, dist_ctx):
         bh = b.cpu().numpy()
         R = oracle_sample_rows(xh, Wh, bh, problem, M, args.cpu_budget)
         t = time_oracle_rows(xh, Wh, bh, problem, list(range(R)))
-        cpu = {"value": flops * R / M / t / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+        cpu = {"value": 2.0 * R * N * K / t / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
                "kind": "oracle", "sample": f"rows 0..{R - 1} of {M} (full N={N}, K={K}); {t:.1f} s"}
 
     if rank == 0:
@@ -350,7 +398,9 @@ def run_fle(args, name, dist_ctx):
             "config": {"workload": name, "M": M, "K": K, "N": N, "epilogue": problem, "precision": args.precision,
                        "l2": "flushed between steps" if flush else "inputs larger than L2",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "plan": fle.plan_string(M, K, N, desc)},
+                       "plan": fle.plan_string(*plan_shape),
+                       **({"variant": variant, "effective_tflops_of_unpooled_problem":
+                           2.0 * M * N * K * world * args.steps / (total_ms * 1e-3) / 1e12} if variant else {})},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": sampler.summary(),
             "gpu_launches": launches_per_step * args.steps,
         }

@@ -118,6 +118,47 @@ int fle_forward(const float* x, const float* W, const float* b,
                 const fle_epilogue_desc* desc, float* out,
                 void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * fle_pool_weights -- the pooled weights of epilogue (c).
+ *
+ * AvgPool1d(k, stride k) over the output features commutes with the Linear
+ * map: the mean of k consecutive outputs is one output of a Linear whose
+ * weight row is the mean of those k weight rows (page "Kimi-K2.6 l2_p98",
+ * its derivation of pre-averaged weights and biases, checked there on a
+ * 2-feature example).  This writes
+ *   W_pooled[j][:] = mean_{t<k} W[j*k + t][:],  b_pooled[j] = mean_{t<k} b[j*k + t]
+ * for j < P = N / pool_k (trailing N mod k rows are unused, as the pool
+ * ignores them).  Then fle_forward(x, W_pooled, b_pooled, M, K, P, desc with
+ * pool_k = pool_stride = 1, out, ...) gives the same out [M] as the
+ * unpooled epilogue (c) call, up to rounding, with a GEMM P/N as large.
+ * W_pooled can be kept and reused while W is unchanged.
+ *
+ *   W        device fp32 [N,K], 16-byte aligned, K % 4 == 0
+ *   b        device fp32 [N] or NULL (then b_pooled is not written)
+ *   pool_k   1, 2, 4, 8, 16 or 32; N >= pool_k
+ *   W_pooled device fp32 [P,K], 16-byte aligned, caller-owned
+ *   b_pooled device fp32 [P] (required when b is not NULL)
+ * Stream-ordered; returns FLE_OK or an argument / CUDA error.
+ */
+int fle_pool_weights(const float* W, const float* b, int64_t N, int64_t K, int32_t pool_k,
+                     float* W_pooled, float* b_pooled, void* stream);
+
+/* Workspace bytes for fle_forward_pooled (pooled weights + the GEMM's own). */
+size_t fle_workspace_size_pooled(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* desc);
+
+/*
+ * fle_forward_pooled -- epilogue (c) by pooled weights in one call: pools W
+ * and b into the workspace (fle_pool_weights), then runs the P/N-times
+ * smaller fused GEMM with the GELU, scale and row-max epilogue.  Same
+ * arguments and result as fle_forward with desc->kind ==
+ * FLE_EPI_AVGPOOL_GELU_SCALE_ROWMAX (FLE_ERR_DESC for other kinds); the
+ * workspace must hold fle_workspace_size_pooled() bytes.
+ */
+int fle_forward_pooled(const float* x, const float* W, const float* b,
+                       int64_t M, int64_t K, int64_t N,
+                       const fle_epilogue_desc* desc, float* out,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bytes of caller workspace fle_forward needs for these arguments (0 when
  * the chosen schedule needs none).  Returns 0 for invalid arguments too;
  * fle_forward then reports the argument error. */

@@ -16,7 +16,8 @@ import os
 __all__ = [
     "EPI_SCALE_HARDTANH_GELU", "EPI_SWISH_SCALE", "EPI_AVGPOOL_GELU_SCALE_ROWMAX", "EPI_NONE",
     "PREC_3XTF32", "PREC_TF32", "EpilogueDesc", "FleError", "desc_for", "forward",
-    "workspace_size", "device_status", "plan_string", "plan_units", "linear_epilogue", "library_path", "load",
+    "workspace_size", "device_status", "plan_string", "plan_units", "pool_weights",
+    "workspace_size_pooled", "forward_pooled", "linear_epilogue", "library_path", "load",
     "PROBLEMS",
 ]
 
@@ -98,6 +99,12 @@ def load():
     lib.fle_plan_units.argtypes = [i64, i64, i64, ctypes.POINTER(EpilogueDesc), ctypes.c_int, ctypes.c_int,
                                    vp, ctypes.c_int, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
     lib.fle_plan_units.restype = ctypes.c_int
+    lib.fle_pool_weights.argtypes = [vp, vp, i64, i64, ctypes.c_int32, vp, vp, vp]
+    lib.fle_pool_weights.restype = ctypes.c_int
+    lib.fle_workspace_size_pooled.argtypes = [i64, i64, i64, ctypes.POINTER(EpilogueDesc)]
+    lib.fle_workspace_size_pooled.restype = sz
+    lib.fle_forward_pooled.argtypes = [vp, vp, vp, i64, i64, i64, ctypes.POINTER(EpilogueDesc), vp, vp, sz, vp]
+    lib.fle_forward_pooled.restype = ctypes.c_int
     lib.fle_test_bounded_wait.argtypes = [ctypes.c_uint32, vp]
     lib.fle_test_bounded_wait.restype = ctypes.c_int
     _lib = lib
@@ -209,6 +216,43 @@ def forward(x, W, b, out, desc: EpilogueDesc, workspace=None, workspace_bytes: i
                          _ptr(workspace), int(workspace_bytes), _stream_handle(stream))
     if st != FLE_OK:
         raise FleError(st, "fle_forward")
+
+
+def pool_weights(W, b, pool_k: int = 16, W_pooled=None, b_pooled=None, stream=None):
+    """fle_pool_weights: (W_pooled [N/k, K], b_pooled [N/k] or None)."""
+    import torch
+    N, K = W.shape
+    P = N // pool_k
+    if W_pooled is None:
+        W_pooled = torch.empty(P, K, dtype=torch.float32, device=W.device)
+    if b is not None and b_pooled is None:
+        b_pooled = torch.empty(P, dtype=torch.float32, device=W.device)
+    st = load().fle_pool_weights(_ptr(W), _ptr(b), N, K, int(pool_k), _ptr(W_pooled),
+                                 _ptr(b_pooled) if b is not None else None, _stream_handle(stream))
+    if st != FLE_OK:
+        raise FleError(st, "fle_pool_weights")
+    return W_pooled, (b_pooled if b is not None else None)
+
+
+def workspace_size_pooled(M: int, K: int, N: int, desc: EpilogueDesc) -> int:
+    return int(load().fle_workspace_size_pooled(M, K, N, ctypes.byref(desc)))
+
+
+def forward_pooled(x, W, b, out, desc: EpilogueDesc, workspace=None, workspace_bytes: int | None = None,
+                   stream=None) -> None:
+    """fle_forward_pooled: epilogue (c) through pooled weights in one call."""
+    M, K = x.shape
+    N = W.shape[0]
+    _check_tensor("x", x, (M, K))
+    _check_tensor("W", W, (N, K))
+    _check_tensor("b", b, (N,))
+    _check_tensor("out", out, (M,))
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load().fle_forward_pooled(_ptr(x), _ptr(W), _ptr(b), M, K, N, ctypes.byref(desc), _ptr(out),
+                                   _ptr(workspace), int(workspace_bytes), _stream_handle(stream))
+    if st != FLE_OK:
+        raise FleError(st, "fle_forward_pooled")
 
 
 def linear_epilogue(x, W, b, problem: str = "scale_hardtanh_gelu", precision: str = "tf32",

@@ -510,6 +510,74 @@ int fle_plan_units(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, 
     return FLE_OK;
 }
 
+int fle_pool_weights(const float* W, const float* b, int64_t N, int64_t K, int32_t pool_k, float* W_pooled,
+                     float* b_pooled, void* stream) {
+    if (!is_pow2_upto32(pool_k)) return FLE_ERR_DESC;
+    const int64_t lim = (int64_t(1) << 31);
+    if (N < pool_k || K < 0 || N >= lim || K >= lim) return FLE_ERR_SHAPE;
+    if (K % 4 != 0) return FLE_ERR_ALIGN;
+    const int64_t P = N / pool_k;
+    if (K > 0 && (!W || !W_pooled)) return FLE_ERR_NULL;
+    if (b && !b_pooled) return FLE_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(W_pooled)) & 15u) return FLE_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(b) | reinterpret_cast<uintptr_t>(b_pooled)) & 3u) return FLE_ERR_ALIGN;
+    DeviceInfo di;
+    int st = device_info(&di);
+    if (st != FLE_OK) return st;
+    const int64_t n = std::max<int64_t>(P * (K / 4), P);
+    const int threads = 256;
+    fle::fle_pool_weights_kernel<<<static_cast<unsigned>((n + threads - 1) / threads), threads, 0,
+                                   static_cast<cudaStream_t>(stream)>>>(W, b, P, K, pool_k, W_pooled, b_pooled);
+    return cudaGetLastError() == cudaSuccess ? FLE_OK : FLE_ERR_CUDA;
+}
+
+namespace {
+// The pool-folded call: desc with the pool replaced by pool_k = 1 on the
+// pooled weights.
+fle_epilogue_desc folded_desc(const fle_epilogue_desc* d) {
+    fle_epilogue_desc f = *d;
+    f.pool_k = 1;
+    f.pool_stride = 1;
+    return f;
+}
+size_t pooled_weight_bytes(int64_t P, int64_t K) {
+    return ((static_cast<size_t>(P) * K * sizeof(float) + 255) & ~size_t(255)) +
+           ((static_cast<size_t>(P) * sizeof(float) + 255) & ~size_t(255));
+}
+}  // namespace
+
+size_t fle_workspace_size_pooled(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d) {
+    if (check_desc(d) != FLE_OK || check_shape(M, K, N, d) != FLE_OK) return 0;
+    if (d->kind != FLE_EPI_AVGPOOL_GELU_SCALE_ROWMAX || M == 0) return 0;
+    const int64_t P = N / d->pool_k;
+    const fle_epilogue_desc f = folded_desc(d);
+    return pooled_weight_bytes(P, K) + fle_workspace_size(M, K, P, &f);
+}
+
+int fle_forward_pooled(const float* x, const float* W, const float* b, int64_t M, int64_t K, int64_t N,
+                       const fle_epilogue_desc* d, float* out, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+    int st = check_desc(d);
+    if (st != FLE_OK) return st;
+    if (d->kind != FLE_EPI_AVGPOOL_GELU_SCALE_ROWMAX) return FLE_ERR_DESC;
+    st = check_shape(M, K, N, d);
+    if (st != FLE_OK) return st;
+    if (M == 0) return FLE_OK;
+    const int64_t P = N / d->pool_k;
+    const size_t need = fle_workspace_size_pooled(M, K, N, d);
+    if (!workspace || workspace_bytes < need) return FLE_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FLE_ERR_ALIGN;
+    char* ws = static_cast<char*>(workspace);
+    float* Wp = reinterpret_cast<float*>(ws);
+    float* bp = reinterpret_cast<float*>(ws + ((static_cast<size_t>(P) * K * sizeof(float) + 255) & ~size_t(255)));
+    const size_t pw = pooled_weight_bytes(P, K);
+    if (K == 0) return fle_forward(x, W, b, M, K, N, d, out, nullptr, 0, stream);  // out = epilogue(b)
+    st = fle_pool_weights(W, b, N, K, d->pool_k, Wp, b ? bp : nullptr, stream);
+    if (st != FLE_OK) return st;
+    const fle_epilogue_desc f = folded_desc(d);
+    return fle_forward(x, Wp, b ? bp : nullptr, M, K, P, &f, out, ws + pw, workspace_bytes - pw, stream);
+}
+
 int fle_device_status(void* stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FLE_ERR_CUDA;
     unsigned h[4] = {0, 0, 0, 0};

@@ -701,6 +701,36 @@ __global__ void fle_prep_kernel(float* fill, int64_t n_fill, unsigned* counters,
     if (counters != nullptr && i < n_counters) counters[i] = 0u;
 }
 
+// Pooled weights for epilogue (c): AvgPool1d(k, stride k) over the output
+// features commutes with the Linear map, so the mean of k consecutive outputs
+// equals one output of the Linear whose weight row is the mean of the k
+// weight rows (and likewise for the bias).  Wp[j][:] = mean_t W[j*k + t][:],
+// bp[j] = mean_t b[j*k + t], for j < P.  Each thread sums k float4 rows in
+// order t = 0..k-1 and scales by 1/k (exact: k is a power of two).  K % 4 == 0.
+__global__ void fle_pool_weights_kernel(const float* __restrict__ W, const float* __restrict__ b,
+                                        int64_t P, int64_t K, int k, float* __restrict__ Wp,
+                                        float* __restrict__ bp) {
+    const int64_t kv = K / 4;
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const float inv_k = 1.0f / static_cast<float>(k);
+    if (i < P * kv) {
+        const int64_t j = i / kv;
+        const int64_t c = i - j * kv;
+        const float4* src = reinterpret_cast<const float4*>(W) + (j * k) * kv + c;
+        float4 acc = __ldcs(src);
+        for (int t = 1; t < k; ++t) {
+            const float4 w = __ldcs(src + t * kv);
+            acc.x += w.x; acc.y += w.y; acc.z += w.z; acc.w += w.w;
+        }
+        reinterpret_cast<float4*>(Wp)[i] = make_float4(acc.x * inv_k, acc.y * inv_k, acc.z * inv_k, acc.w * inv_k);
+    }
+    if (b != nullptr && bp != nullptr && i < P) {
+        float acc = b[i * k];
+        for (int t = 1; t < k; ++t) acc += b[i * k + t];
+        bp[i] = acc * inv_k;
+    }
+}
+
 // Test hook: one thread waits on a barrier nothing arrives on.
 __global__ void fle_bounded_wait_test_kernel(uint64_t timeout_ns) {
     __shared__ __align__(8) uint64_t bar;
