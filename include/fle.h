@@ -234,6 +234,16 @@ int fle_version(void);
  */
 int fle_test_bounded_wait(uint32_t timeout_us, void* stream);
 
+/*
+ * Test hook for the epilogue's scalar math: out[i] = f(in[i]) for device
+ * arrays of n floats, with f = erf (which = 0), exact-form GELU (1) or
+ * x * sigmoid(x) (2), evaluated either as the fused epilogue evaluates it
+ * (reference = 0) or with CUDA's erff/expf and IEEE division (reference = 1),
+ * so tests can bound the difference.  Stream-ordered.
+ */
+int fle_test_epilogue_math(const float* in, float* out, int64_t n, int32_t which, int32_t reference,
+                           void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -99,6 +99,20 @@ int encode_operand(CUtensorMap* map, const float* base, int64_t rows, int64_t K,
     return r == CUDA_SUCCESS ? FLE_OK : FLE_ERR_CUDA;
 }
 
+// 2-D fp32 output [rows, cols] for epilogue TMA stores: box of 32 columns
+// (128 bytes) by 32 rows, 128-byte swizzle; out-of-range elements are not
+// written.
+int encode_output(CUtensorMap* map, float* base, int64_t rows, int64_t cols) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * sizeof(float)};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FLE_OK : FLE_ERR_CUDA;
+}
+
 bool is_pow2_upto32(int k) { return k == 1 || k == 2 || k == 4 || k == 8 || k == 16 || k == 32; }
 
 int check_desc(const fle_epilogue_desc* d) {
@@ -236,9 +250,9 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
 }
 
 template <int BN, int PREC, bool SWAP>
-cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const KParams& p, int grid,
-                        cudaStream_t st) {
-    using C = fle::Cfg<BN, PREC>;
+cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to, const KParams& p,
+                        int grid, cudaStream_t st) {
+    using C = fle::Cfg<BN, PREC, SWAP>;
     auto kern = fle::fle_gemm_kernel<BN, PREC, SWAP>;
     static bool attr_set[kMaxDevices] = {};
     int dev = 0;
@@ -248,12 +262,12 @@ cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const KPar
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    kern<<<grid, fle::kThreads, C::kSmemBytes, st>>>(ta, tb, p);
+    kern<<<grid, fle::kThreads, C::kSmemBytes, st>>>(ta, tb, to, p);
     return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const KParams& p, int pairs,
-                             cudaStream_t st) {
+cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to, const KParams& p,
+                             int pairs, cudaStream_t st) {
     // max_active_pairs() set the kernel's shared-memory attribute when the
     // device was probed.
     cudaLaunchConfig_t cfg = {};
@@ -268,29 +282,29 @@ cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, fle::fle_gemm_pair_kernel<fle::kPrecTF32>, ta, tb, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, fle::fle_gemm_pair_kernel<fle::kPrecTF32>, ta, tb, to, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
-cudaError_t dispatch(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const KParams& p,
-                     cudaStream_t st) {
+cudaError_t dispatch(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
+                     const KParams& p, cudaStream_t st) {
     const bool tf32 = pl.prec == fle::kPrecTF32;
-    if (pl.pair) return launch_gemm_pair(ta, tb, p, pl.grid, st);
+    if (pl.pair) return launch_gemm_pair(ta, tb, to, p, pl.grid, st);
     if (!pl.swap) {
-        if (tf32 && pl.bn == 256) return launch_gemm<256, fle::kPrecTF32, false>(ta, tb, p, pl.grid, st);
-        if (!tf32 && pl.bn == 128) return launch_gemm<128, fle::kPrec3xTF32, false>(ta, tb, p, pl.grid, st);
+        if (tf32 && pl.bn == 256) return launch_gemm<256, fle::kPrecTF32, false>(ta, tb, to, p, pl.grid, st);
+        if (!tf32 && pl.bn == 128) return launch_gemm<128, fle::kPrec3xTF32, false>(ta, tb, to, p, pl.grid, st);
     } else {
         switch (pl.bn) {
             case 32:
-                return tf32 ? launch_gemm<32, fle::kPrecTF32, true>(ta, tb, p, pl.grid, st)
-                            : launch_gemm<32, fle::kPrec3xTF32, true>(ta, tb, p, pl.grid, st);
+                return tf32 ? launch_gemm<32, fle::kPrecTF32, true>(ta, tb, to, p, pl.grid, st)
+                            : launch_gemm<32, fle::kPrec3xTF32, true>(ta, tb, to, p, pl.grid, st);
             case 64:
-                return tf32 ? launch_gemm<64, fle::kPrecTF32, true>(ta, tb, p, pl.grid, st)
-                            : launch_gemm<64, fle::kPrec3xTF32, true>(ta, tb, p, pl.grid, st);
+                return tf32 ? launch_gemm<64, fle::kPrecTF32, true>(ta, tb, to, p, pl.grid, st)
+                            : launch_gemm<64, fle::kPrec3xTF32, true>(ta, tb, to, p, pl.grid, st);
             case 128:
-                return tf32 ? launch_gemm<128, fle::kPrecTF32, true>(ta, tb, p, pl.grid, st)
-                            : launch_gemm<128, fle::kPrec3xTF32, true>(ta, tb, p, pl.grid, st);
+                return tf32 ? launch_gemm<128, fle::kPrecTF32, true>(ta, tb, to, p, pl.grid, st)
+                            : launch_gemm<128, fle::kPrec3xTF32, true>(ta, tb, to, p, pl.grid, st);
             default: break;
         }
     }
@@ -438,7 +452,15 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
         p.counters = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + pl.partial_bytes);
     }
 
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, to;
+    std::memset(&to, 0, sizeof to);
+    // Direct-layout elementwise kinds store through TMA when the output rows
+    // are 16-byte multiples and the base is 16-byte aligned.
+    p.tma_out = (!pl.swap && !pool && N % 4 == 0 && (reinterpret_cast<uintptr_t>(out) & 15u) == 0) ? 1 : 0;
+    if (p.tma_out) {
+        st = encode_output(&to, out, M, N);
+        if (st != FLE_OK) return st;
+    }
     const float* A = pl.swap ? W : x;
     const float* B = pl.swap ? x : W;
     st = encode_operand(&ta, A, p.Ma, K, fle::kBM);
@@ -461,7 +483,7 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
             pool ? out : nullptr, pool ? M : 0, p.counters, n_counters);
         if (cudaGetLastError() != cudaSuccess) return FLE_ERR_CUDA;
     }
-    if (dispatch(pl, ta, tb, p, s) != cudaSuccess) return FLE_ERR_CUDA;
+    if (dispatch(pl, ta, tb, to, p, s) != cudaSuccess) return FLE_ERR_CUDA;
     if (sync_check_enabled()) return fle_device_status(stream);
     return FLE_OK;
 }
@@ -590,6 +612,24 @@ int fle_device_status(void* stream) {
         return static_cast<int>(h[0]);
     }
     return FLE_OK;
+}
+
+int fle_test_epilogue_math(const float* in, float* out, int64_t n, int32_t which, int32_t reference,
+                           void* stream) {
+    if (!in || !out) return FLE_ERR_NULL;
+    if (n < 0 || which < 0 || which > 2) return FLE_ERR_SHAPE;
+    DeviceInfo di;
+    int st = device_info(&di);
+    if (st != FLE_OK) return st;
+    if (n == 0) return FLE_OK;
+    const int threads = 256;
+    const unsigned blocks = static_cast<unsigned>((n + threads - 1) / threads);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (reference)
+        fle::fle_math_reference_kernel<<<blocks, threads, 0, s>>>(in, out, n, which);
+    else
+        fle::fle_math_probe_kernel<<<blocks, threads, 0, s>>>(in, out, n, which);
+    return cudaGetLastError() == cudaSuccess ? FLE_OK : FLE_ERR_CUDA;
 }
 
 int fle_test_bounded_wait(uint32_t timeout_us, void* stream) {

@@ -40,6 +40,8 @@ constexpr int kBM = 128;           // MMA M: rows of operand A per tile
 constexpr int kBK = 32;            // fp32 per k-block = one 128-byte swizzled row
 constexpr int kUmmaK = 8;          // K of one tcgen05.mma kind::tf32
 constexpr int kThreads = 384;
+constexpr int kEpiWarps = 8;                 // warps 4..11
+constexpr int kEpiTileBytes = 32 * 32 * 4;   // one warp's 32 x 32 fp32 block
 constexpr int kSmemStageBudget = 229376;  // bytes of shared memory for stages (224 KB)
 
 enum : int { kEpiHardtanhGelu = 0, kEpiSwish = 1, kEpiPoolMax = 2, kEpiNone = 3 };
@@ -70,6 +72,7 @@ struct KParams {
     int64_t pool_limit;     // columns covered by complete pool windows
     int vec_out;            // out 16-byte aligned and N % 4 == 0
     int vec_bias;           // bias 16-byte aligned
+    int tma_out;            // direct layout: write out through TMA tile stores
     uint64_t timeout_ns;
 };
 
@@ -141,29 +144,52 @@ __host__ __device__ __forceinline__ int sk_slot_of(int c, int64_t tsk, int64_t s
     return (tsk == gb / num_kb) ? 0 : 1;
 }
 
-template <int BN, int PREC>
+template <int BN, int PREC, bool SWAP>
 struct Cfg {
     static constexpr int kABytes = kBM * kBK * 4;
     static constexpr int kBBytes = BN * kBK * 4;
     static constexpr int kLoadBytes = kABytes + kBBytes;            // TMA bytes per stage
     static constexpr int kStageBytes = kLoadBytes * (PREC == kPrec3xTF32 ? 2 : 1);
-    static constexpr int kStagesRaw = kSmemStageBudget / kStageBytes;
+    // direct layout: one 32 x 32 fp32 staging tile per epilogue warp for TMA stores
+    static constexpr int kEpiStageBytes = SWAP ? 0 : kEpiWarps * kEpiTileBytes;
+    static constexpr int kStagesRaw = (kSmemStageBudget - kEpiStageBytes) / kStageBytes;
     static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
     static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                     : (2 * BN <= 256) ? 256 : 512;
     // barriers: full, conv, empty per stage; accf, acce per buffer; drain
     static constexpr int kNumBars = 3 * kStages + 4 + 1;
-    static constexpr int kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + kNumBars * 8 + 32;
+    static constexpr int kSmemBytes =
+        1024 /*align slack*/ + kStages * kStageBytes + kEpiStageBytes + kNumBars * 8 + 32;
     static_assert(kStages >= 2, "need at least two stages");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128 is a multiple of 16 in [16,256]");
     static_assert(kABytes % 1024 == 0 && kBBytes % 1024 == 0, "tiles must keep 1024-byte alignment");
+    static_assert(kSmemBytes <= 232448, "exceeds 227 KB of shared memory per block");
 };
 
 // ----------------------------------------------------------------------------
 // Epilogue math
 // ----------------------------------------------------------------------------
+// erf(x) by Abramowitz & Stegun, Handbook of Mathematical Functions, formula
+// 7.1.26 (Hastings' rational approximation): for x >= 0,
+//   erf(x) = 1 - (a1 s + a2 s^2 + a3 s^3 + a4 s^4 + a5 s^5) exp(-x^2),
+//   s = 1 / (1 + p x),  |error| <= 1.5e-7,
+// extended to x < 0 by oddness.  One reciprocal and one exponential instead
+// of a long polynomial chain: the epilogue runs it once per output element.
+__device__ __forceinline__ float erf_as7126(float x) {
+    const float ax = fabsf(x);
+    const float s = __fdividef(1.0f, fmaf(0.3275911f, ax, 1.0f));
+    float poly = fmaf(s, 1.061405429f, -1.453152027f);
+    poly = fmaf(s, poly, 1.421413741f);
+    poly = fmaf(s, poly, -0.284496736f);
+    poly = fmaf(s, poly, 0.254829592f);
+    poly *= s;
+    const float r = fmaf(-poly, __expf(-ax * ax), 1.0f);
+    return copysignf(r, x);
+}
+
+// Exact-form GELU: t * Phi(t) = t * (1 + erf(t / sqrt 2)) / 2.
 __device__ __forceinline__ float gelu_erf(float t) {
-    return t * 0.5f * (1.0f + erff(t * 0.70710678118654752440f));
+    return t * 0.5f * (1.0f + erf_as7126(t * 0.70710678118654752440f));
 }
 
 template <int KIND>
@@ -173,7 +199,9 @@ __device__ __forceinline__ float epi_apply(float y, const KParams& p) {
         t = fminf(fmaxf(t, p.clamp_lo), p.clamp_hi);
         return gelu_erf(t);
     } else if constexpr (KIND == kEpiSwish) {
-        return (y / (1.0f + expf(-y))) * p.scale;
+        // y * sigmoid(y); for y -> -inf, exp(-y) overflows to inf and the
+        // quotient goes to 0 (the limit), never NaN.
+        return __fdividef(y, 1.0f + __expf(-y)) * p.scale;
     } else {
         return y;
     }
@@ -207,13 +235,43 @@ __device__ __forceinline__ void load_bias32(const KParams& p, int64_t n0, float 
     }
 }
 
+// Where a direct-layout epilogue warp sends its finished 32 x 32 block: through
+// its swizzled shared-memory staging tile and one TMA tile store (tmap set),
+// or with plain per-thread stores.
+struct EpiOut {
+    const CUtensorMap* tmap;  // nullptr: plain stores
+    float* stage;             // this warp's staging tile, 1024-byte aligned
+    uint32_t stage_u32;
+    int64_t row0;             // first output row of this warp's 32 rows
+};
+
 // Direct layout, elementwise kinds: this thread holds row m, columns n0..n0+31.
 template <int KIND>
-__device__ __forceinline__ void epi_store_direct(const KParams& p, int64_t m, int64_t n0, float (&v)[32]) {
+__device__ __forceinline__ void epi_store_direct(const KParams& p, const EpiOut& eo, int64_t m, int64_t n0,
+                                                 float (&v)[32]) {
     float bv[32];
     load_bias32(p, n0, bv);
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = epi_apply<KIND>(v[j] + bv[j], p);
+    if (eo.tmap != nullptr) {
+        // Row r of the block goes to staging row r; its eight 16-byte pieces
+        // are placed at piece index (i ^ (r % 8)), the 128-byte swizzle the
+        // tensor map was encoded with, so the writes hit distinct banks.
+        const int lane = threadIdx.x & 31;
+        if (lane == 0) bulk_wait_read_all();  // the previous block has left this tile
+        __syncwarp();
+        float4* row = reinterpret_cast<float4*>(eo.stage + lane * 32);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            row[i ^ (lane & 7)] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(eo.tmap, eo.stage_u32, static_cast<int32_t>(n0), static_cast<int32_t>(eo.row0));
+            bulk_commit_group();
+        }
+        return;
+    }
     if (m >= p.M) return;
     float* dst = p.out + m * p.N + n0;
     if (p.vec_out && n0 + 32 <= p.N) {
@@ -265,15 +323,15 @@ __device__ __forceinline__ void epi_store_swapped(const KParams& p, int64_t n, i
 // windows are folded into `best`; epi_finish then combines it across CTAs.
 template <bool SWAP, int BN>
 __device__ __forceinline__ void epi_chunk(const KParams& p, const Unit& u, int r, int c, float (&v)[32],
-                                          float& best) {
+                                          float& best, const EpiOut& eo) {
     if constexpr (!SWAP) {
         const int64_t m = static_cast<int64_t>(u.ta) * kBM + r;
         const int64_t n0 = static_cast<int64_t>(u.tb) * BN + c * 32;
         switch (p.kind) {
-            case kEpiHardtanhGelu: epi_store_direct<kEpiHardtanhGelu>(p, m, n0, v); break;
-            case kEpiSwish: epi_store_direct<kEpiSwish>(p, m, n0, v); break;
+            case kEpiHardtanhGelu: epi_store_direct<kEpiHardtanhGelu>(p, eo, m, n0, v); break;
+            case kEpiSwish: epi_store_direct<kEpiSwish>(p, eo, m, n0, v); break;
             case kEpiPoolMax: epi_pool_direct(p, n0, v, best); break;
-            default: epi_store_direct<kEpiNone>(p, m, n0, v); break;
+            default: epi_store_direct<kEpiNone>(p, eo, m, n0, v); break;
         }
     } else {
         const int64_t n = static_cast<int64_t>(u.ta) * kBM + r;
@@ -305,8 +363,8 @@ __device__ __forceinline__ void epilogue_bar_sync() {
 template <int BN, int PREC, bool SWAP>
 __global__ void __launch_bounds__(kThreads, 1)
 fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const KParams p) {
-    using C = Cfg<BN, PREC>;
+                const __grid_constant__ CUtensorMap tmOut, const KParams p) {
+    using C = Cfg<BN, PREC, SWAP>;
     constexpr int S = C::kStages;
     constexpr uint32_t kIdesc = idesc_tf32(kBM, BN);
     // k-blocks per TMEM accumulation chain (see the epilogue role)
@@ -315,7 +373,8 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+    uint8_t* epi_stage = smem + S * C::kStageBytes;  // C::kEpiStageBytes
+    uint64_t* bars = reinterpret_cast<uint64_t*>(epi_stage + C::kEpiStageBytes);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
@@ -501,6 +560,11 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         const int q = warp & 3;
         const int half = (warp - 4) >> 2;
         const int r = q * 32 + lane;  // tile row = TMEM lane of this thread
+        EpiOut eo;
+        eo.tmap = (!SWAP && p.tma_out) ? &tmOut : nullptr;
+        eo.stage = reinterpret_cast<float*>(epi_stage + (SWAP ? 0 : (warp - 4) * kEpiTileBytes));
+        eo.stage_u32 = smem_u32(eo.stage);
+        eo.row0 = 0;
         constexpr int kChunks = BN / 32;
         constexpr int kHalf = (kChunks + 1) / 2;  // chunks per half
         const int c_lo = half * kHalf;
@@ -522,6 +586,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             const int64_t cols_left = (SWAP ? p.M : p.N) - static_cast<int64_t>(u.tb) * BN;
             const int nchunks = static_cast<int>(cols_left >= BN ? kChunks : (cols_left + 31) / 32);
             const int mine = nchunks - c_lo < 0 ? 0 : (nchunks - c_lo > kHalf ? kHalf : nchunks - c_lo);
+            eo.row0 = static_cast<int64_t>(u.ta) * kBM + q * 32;
 
             auto wait_acc = [&]() -> bool {
                 int got = 0;
@@ -581,7 +646,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     {                                                        \
         float v[32];                                         \
         FLE_LOAD_ACC(lc, v);                                 \
-        epi_chunk<SWAP, BN>(p, u, r, c_lo + (lc), v, best);  \
+        epi_chunk<SWAP, BN>(p, u, r, c_lo + (lc), v, best, eo);  \
     }
                 if constexpr (kRegAcc) {
 #pragma unroll
@@ -638,17 +703,37 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         float v[32];
 #pragma unroll
                         for (int j = 0; j < 32; ++j) v[j] = 0.0f;
-                        for (int cc = first; cc <= last; ++cc) {
+                        // Contributors in CTA order; loads of up to three
+                        // contributors are in flight together.
+                        auto src_of = [&](int cc) {
                             const int sl = sk_slot_of(cc, tsk, p.sk_iters, p.sk_grid, p.num_kb);
-                            const float* src = p.ws + static_cast<size_t>(2 * cc + sl) * kBM * BN +
-                                               static_cast<size_t>(c * 32) * kBM + r;
-                            float t[32];
+                            return p.ws + static_cast<size_t>(2 * cc + sl) * kBM * BN +
+                                   static_cast<size_t>(c * 32) * kBM + r;
+                        };
+                        int cc = first;
+                        for (; cc + 2 <= last; cc += 3) {
+                            const float* s0 = src_of(cc);
+                            const float* s1 = src_of(cc + 1);
+                            const float* s2 = src_of(cc + 2);
+                            float t0[32], t1[32], t2[32];
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) t[j] = __ldcg(src + j * kBM);
+                            for (int j = 0; j < 32; ++j) {
+                                t0[j] = __ldcg(s0 + j * kBM);
+                                t1[j] = __ldcg(s1 + j * kBM);
+                                t2[j] = __ldcg(s2 + j * kBM);
+                            }
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) v[j] += t[j];
+                            for (int j = 0; j < 32; ++j) v[j] = ((v[j] + t0[j]) + t1[j]) + t2[j];
                         }
-                        epi_chunk<SWAP, BN>(p, u, r, c, v, best);
+                        for (; cc <= last; ++cc) {
+                            const float* s0 = src_of(cc);
+                            float t0[32];
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) t0[j] = __ldcg(s0 + j * kBM);
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] += t0[j];
+                        }
+                        epi_chunk<SWAP, BN>(p, u, r, c, v, best, eo);
                     }
                     epi_finish<SWAP>(p, u, r, best);
                     if (threadIdx.x == 128) p.counters[tsk] = 0u;
@@ -658,6 +743,8 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         }
     }
 
+    // Epilogue TMA stores read the staging tiles until they complete.
+    if (warp >= 4 && lane == 0) bulk_wait_all();
     tc_fence_before_sync();
     __syncthreads();
     if (warp == 1) {
@@ -729,6 +816,25 @@ __global__ void fle_pool_weights_kernel(const float* __restrict__ W, const float
         for (int t = 1; t < k; ++t) acc += b[i * k + t];
         bp[i] = acc * inv_k;
     }
+}
+
+// Test hook: the epilogue's scalar functions on n inputs (kind 0: erf,
+// 1: GELU, 2: swish with scale 1), for checks against CUDA's erff/expf.
+__global__ void fle_math_probe_kernel(const float* in, float* out, int64_t n, int which) {
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    const float v = in[i];
+    if (which == 0) out[i] = erf_as7126(v);
+    else if (which == 1) out[i] = gelu_erf(v);
+    else out[i] = __fdividef(v, 1.0f + __expf(-v));
+}
+__global__ void fle_math_reference_kernel(const float* in, float* out, int64_t n, int which) {
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    const float v = in[i];
+    if (which == 0) out[i] = erff(v);
+    else if (which == 1) out[i] = v * 0.5f * (1.0f + erff(v * 0.70710678118654752440f));
+    else out[i] = v / (1.0f + expf(-v));
 }
 
 // Test hook: one thread waits on a barrier nothing arrives on.

@@ -27,17 +27,19 @@ struct PairCfg {
     static constexpr int kABytes = kBM * kBK * 4;          // this CTA's 128 A rows
     static constexpr int kBBytes = (kPairBN / 2) * kBK * 4;  // this CTA's 128 B rows
     static constexpr int kLoadBytes = kABytes + kBBytes;
-    static constexpr int kStages = 7;  // 224 KB of stages; the tile needs no other shared memory
+    static constexpr int kEpiStageBytes = kEpiWarps * kEpiTileBytes;  // TMA-store staging
+    static constexpr int kStages = (kSmemStageBudget - kEpiStageBytes) / kLoadBytes;  // 6
     static constexpr int kTmemCols = 512;                    // 2 accumulator buffers x 256 columns
     // full, empty per stage; accf, acce per buffer; drain; exit
     static constexpr int kNumBars = 2 * kStages + 4 + 2;
-    static constexpr int kSmemBytes = 1024 + kStages * kLoadBytes + kNumBars * 8 + 32;
+    static constexpr int kSmemBytes = 1024 + kStages * kLoadBytes + kEpiStageBytes + kNumBars * 8 + 32;
+    static_assert(kSmemBytes <= 232448, "exceeds 227 KB of shared memory per block");
 };
 
 template <int PREC>
 __global__ void __launch_bounds__(kThreads, 1)
 fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const KParams p) {
+                     const __grid_constant__ CUtensorMap tmOut, const KParams p) {
     static_assert(PREC == kPrecTF32, "CTA-pair kernel: single-pass TF32");
     using C = PairCfg;
     constexpr int S = C::kStages;
@@ -46,7 +48,8 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kLoadBytes);
+    uint8_t* epi_stage = smem + S * C::kLoadBytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(epi_stage + C::kEpiStageBytes);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
@@ -179,6 +182,10 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         const int r = q * 32 + lane;
         constexpr int kHalf = kPairBN / 32 / 2;  // chunks per half
         const int c_lo = half * kHalf;
+        EpiOut eo;
+        eo.tmap = p.tma_out ? &tmOut : nullptr;
+        eo.stage = reinterpret_cast<float*>(epi_stage + (warp - 4) * kEpiTileBytes);
+        eo.stage_u32 = smem_u32(eo.stage);
         int buf = 0;
         uint32_t acc_phase = 0;
         Sched sc;
@@ -198,6 +205,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             // This CTA's 128 rows of the pair tile, as a 128-row tile index.
             Unit uh = u;
             uh.ta = 2 * u.ta + static_cast<int>(rank);
+            eo.row0 = static_cast<int64_t>(uh.ta) * kBM + q * 32;
             auto release_acc = [&]() {
                 tc_fence_before_sync();
                 __syncwarp();
@@ -212,7 +220,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 for (int lc = 0; lc < mine; ++lc) {
                     float v[32];
                     tmem_ld32_wait(t_acc + (c_lo + lc) * 32, v);
-                    epi_chunk<false, kPairBN>(p, uh, r, c_lo + lc, v, best);
+                    epi_chunk<false, kPairBN>(p, uh, r, c_lo + lc, v, best, eo);
                 }
                 epi_finish<false>(p, uh, r, best);
                 release_acc();
@@ -248,17 +256,37 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                         float v[32];
 #pragma unroll
                         for (int j = 0; j < 32; ++j) v[j] = 0.0f;
-                        for (int cc = first; cc <= last; ++cc) {
+                        // Contributors in CTA order; loads of up to three
+                        // contributors are in flight together.
+                        auto src_of = [&](int cc) {
                             const int sl = sk_slot_of(cc, tsk, p.sk_iters, p.sk_grid, p.num_kb);
-                            const float* src = p.ws + static_cast<size_t>(2 * (2 * cc + rank) + sl) * kBM * kPairBN +
-                                               static_cast<size_t>(c * 32) * kBM + r;
-                            float t[32];
+                            return p.ws + static_cast<size_t>(2 * (2 * cc + rank) + sl) * kBM * kPairBN +
+                                   static_cast<size_t>(c * 32) * kBM + r;
+                        };
+                        int cc = first;
+                        for (; cc + 2 <= last; cc += 3) {
+                            const float* s0 = src_of(cc);
+                            const float* s1 = src_of(cc + 1);
+                            const float* s2 = src_of(cc + 2);
+                            float t0[32], t1[32], t2[32];
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) t[j] = __ldcg(src + j * kBM);
+                            for (int j = 0; j < 32; ++j) {
+                                t0[j] = __ldcg(s0 + j * kBM);
+                                t1[j] = __ldcg(s1 + j * kBM);
+                                t2[j] = __ldcg(s2 + j * kBM);
+                            }
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) v[j] += t[j];
+                            for (int j = 0; j < 32; ++j) v[j] = ((v[j] + t0[j]) + t1[j]) + t2[j];
                         }
-                        epi_chunk<false, kPairBN>(p, uh, r, c, v, best);
+                        for (; cc <= last; ++cc) {
+                            const float* s0 = src_of(cc);
+                            float t0[32];
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) t0[j] = __ldcg(s0 + j * kBM);
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] += t0[j];
+                        }
+                        epi_chunk<false, kPairBN>(p, uh, r, c, v, best, eo);
                     }
                     epi_finish<false>(p, uh, r, best);
                     if (threadIdx.x == 128) *counter = 0u;
@@ -267,6 +295,8 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         }
     }
 
+    // Epilogue TMA stores read the staging tiles until they complete.
+    if (warp >= 4 && lane == 0) bulk_wait_all();
     // Neither CTA may release TMEM or exit while the other can still signal
     // its barriers or (leader) write its TMEM: a bounded two-way handshake.
     tc_fence_before_sync();

@@ -8,6 +8,7 @@ Small shapes (several tiles plus ragged tails, both the direct and the
 swapped operand order) are compared in full; the full-size workloads on a
 seeded sample of whole rows, in the same launch plan the benchmark times.
 """
+import ctypes
 import math
 
 import numpy as np
@@ -61,7 +62,7 @@ def _run(fle, x, W, b, problem, precision):
 
 
 SMALL = [(1, 4, 1), (7, 36, 33), (16, 64, 130), (33, 100, 257), (128, 1024, 1024),
-         (130, 68, 300), (257, 260, 520), (300, 132, 1000)]
+         (130, 68, 300), (257, 260, 520), (300, 132, 1000), (200, 64, 301)]
 PROBLEMS = ["scale_hardtanh_gelu", "swish_scale", "avgpool_gelu_scale_rowmax", "none"]
 
 
@@ -271,3 +272,35 @@ def test_long_k_accuracy_3xtf32(fle, precision):
         out = _run(fle, x, W, b, "none", precision)
         rows = synth.sample_rows(M, 32, seed=2)
         _assert_close(out.cpu().numpy()[rows], _oracle(x, W, b, "none", rows=rows), precision, f"K=32768 {M}x{N}")
+
+
+@pytest.mark.parametrize("which", [0, 1, 2])
+def test_epilogue_math_against_fp64_and_cuda(fle, which):
+    # The epilogue evaluates erf by Abramowitz & Stegun 7.1.26 (|error| <=
+    # 1.5e-7) and the sigmoid with a fast exponential and divide; bound both
+    # against fp64 and against CUDA's erff / expf on a dense grid.
+    from scipy.special import erf as erf64
+    lib = fle.load()
+    lib.fle_test_epilogue_math.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32,
+                                           ctypes.c_int32, ctypes.c_void_p]
+    xs = torch.linspace(-9.0, 9.0, 360001, device="cuda")
+    got = torch.empty_like(xs)
+    cuda_ref = torch.empty_like(xs)
+    assert lib.fle_test_epilogue_math(xs.data_ptr(), got.data_ptr(), xs.numel(), which, 0, None) == 0
+    assert lib.fle_test_epilogue_math(xs.data_ptr(), cuda_ref.data_ptr(), xs.numel(), which, 1, None) == 0
+    torch.cuda.synchronize()
+    x = xs.cpu().numpy().astype(np.float64)
+    g = got.cpu().numpy().astype(np.float64)
+    c = cuda_ref.cpu().numpy().astype(np.float64)
+    if which == 0:
+        exact = erf64(x)
+        bound = 6e-7 * np.ones_like(x)  # A&S bound 1.5e-7 plus fast exp and reciprocal rounding
+    elif which == 1:
+        exact = x * 0.5 * (1 + erf64(x / np.sqrt(2)))
+        bound = 2.5e-7 * np.maximum(1.0, np.abs(x))
+    else:
+        exact = x / (1 + np.exp(-x))
+        bound = 4e-6 * np.maximum(1.0, np.abs(x))
+    assert np.isfinite(g).all()
+    assert np.abs(g - exact).max() <= bound.max() and (np.abs(g - exact) <= bound).all()
+    assert (np.abs(g - c) <= 2 * bound).all()
