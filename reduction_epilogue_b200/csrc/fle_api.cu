@@ -25,19 +25,21 @@ struct DeviceInfo {
     bool probed = false;
     bool ok = false;
     int sms = 0;
-    int pairs = 0;  // co-resident CTA pairs of the pair kernel (0: pair mode unavailable)
+    int pairs = 0;    // co-resident CTA pairs of the TF32 pair kernel (0: unavailable)
+    int pairs3x = 0;  // and of the 3xTF32 pair kernel
 };
 
-// Co-resident 2-CTA clusters of the pair kernel on the current device.
+// Co-resident 2-CTA clusters of a pair kernel on the current device.
+template <int PREC>
 int max_active_pairs() {
-    auto kern = fle::fle_gemm_pair_kernel<fle::kPrecTF32>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, fle::PairCfg::kSmemBytes) !=
-        cudaSuccess)
+    auto kern = fle::fle_gemm_pair_kernel<PREC>;
+    const int smem = fle::PairCfg<PREC>::kSmemBytes;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(fle::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = fle::PairCfg::kSmemBytes;
+    cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
@@ -71,7 +73,8 @@ int device_info(DeviceInfo* out) {
         d.probed = true;
         d.ok = (major == 10 && minor == 0);
         d.sms = sms;
-        d.pairs = d.ok ? max_active_pairs() : 0;
+        d.pairs = d.ok ? max_active_pairs<fle::kPrecTF32>() : 0;
+        d.pairs3x = d.ok ? max_active_pairs<fle::kPrec3xTF32>() : 0;
     }
     if (!d.ok) return FLE_ERR_ARCH;
     if (!g_encode) {
@@ -185,7 +188,7 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
     Plan pl;
     pl.prec = (d->precision == FLE_PREC_3XTF32) ? fle::kPrec3xTF32 : fle::kPrecTF32;
     pl.swap = (M <= 128) && d->kind != FLE_EPI_AVGPOOL_GELU_SCALE_ROWMAX;
-    pl.pair = !pl.swap && pl.prec == fle::kPrecTF32 && M > 128 && pairs > 0 && !pair_disabled();
+    pl.pair = !pl.swap && M > 128 && pairs > 0 && !pair_disabled();
     int tile_m = fle::kBM;
     if (pl.pair) {
         tile_m = fle::kPairBM;
@@ -201,7 +204,9 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
     pl.tiles_b = static_cast<int>((Nb + pl.bn - 1) / pl.bn);
     pl.tiles = pl.tiles_a * pl.tiles_b;
     pl.num_kb = static_cast<int>((K + fle::kBK - 1) / fle::kBK);
-    pl.stages = pl.pair ? fle::PairCfg::kStages : stages_for(pl.bn, pl.prec);
+    pl.stages = pl.pair ? (pl.prec == fle::kPrec3xTF32 ? fle::PairCfg<fle::kPrec3xTF32>::kStages
+                                                       : fle::PairCfg<fle::kPrecTF32>::kStages)
+                        : stages_for(pl.bn, pl.prec);
 
     // The schedule runs over CTAs, or over CTA pairs in pair mode.
     const int64_t T = pl.tiles;
@@ -266,6 +271,7 @@ cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
     return cudaGetLastError();
 }
 
+template <int PREC>
 cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to, const KParams& p,
                              int pairs, cudaStream_t st) {
     // max_active_pairs() set the kernel's shared-memory attribute when the
@@ -273,7 +279,7 @@ cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
     cfg.blockDim = dim3(fle::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = fle::PairCfg::kSmemBytes;
+    cfg.dynamicSmemBytes = fle::PairCfg<PREC>::kSmemBytes;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -282,7 +288,7 @@ cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, fle::fle_gemm_pair_kernel<fle::kPrecTF32>, ta, tb, to, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, fle::fle_gemm_pair_kernel<PREC>, ta, tb, to, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -290,7 +296,9 @@ cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const
 cudaError_t dispatch(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
                      const KParams& p, cudaStream_t st) {
     const bool tf32 = pl.prec == fle::kPrecTF32;
-    if (pl.pair) return launch_gemm_pair(ta, tb, to, p, pl.grid, st);
+    if (pl.pair)
+        return tf32 ? launch_gemm_pair<fle::kPrecTF32>(ta, tb, to, p, pl.grid, st)
+                    : launch_gemm_pair<fle::kPrec3xTF32>(ta, tb, to, p, pl.grid, st);
     if (!pl.swap) {
         if (tf32 && pl.bn == 256) return launch_gemm<256, fle::kPrecTF32, false>(ta, tb, to, p, pl.grid, st);
         if (!tf32 && pl.bn == 128) return launch_gemm<128, fle::kPrec3xTF32, false>(ta, tb, to, p, pl.grid, st);
@@ -375,7 +383,7 @@ size_t fle_workspace_size(int64_t M, int64_t K, int64_t N, const fle_epilogue_de
     if (M == 0 || N == 0 || K == 0) return 0;
     DeviceInfo di;
     if (device_info(&di) != FLE_OK) return 0;
-    return make_plan(M, K, N, d, di.sms, di.pairs).ws_bytes;
+    return make_plan(M, K, N, d, di.sms, d->precision == FLE_PREC_3XTF32 ? di.pairs3x : di.pairs).ws_bytes;
 }
 
 int fle_plan_string(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, char* buf, size_t n) {
@@ -386,7 +394,7 @@ int fle_plan_string(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d,
     DeviceInfo di;
     st = device_info(&di);
     if (st != FLE_OK) return st;
-    return plan_to_string(make_plan(M, K, N, d, di.sms, di.pairs), buf, n);
+    return plan_to_string(make_plan(M, K, N, d, di.sms, d->precision == FLE_PREC_3XTF32 ? di.pairs3x : di.pairs), buf, n);
 }
 
 int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64_t K, int64_t N,
@@ -433,7 +441,7 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
         return cudaGetLastError() == cudaSuccess ? FLE_OK : FLE_ERR_CUDA;
     }
 
-    const Plan pl = make_plan(M, K, N, d, di.sms, di.pairs);
+    const Plan pl = make_plan(M, K, N, d, di.sms, d->precision == FLE_PREC_3XTF32 ? di.pairs3x : di.pairs);
     if (pl.ws_bytes > 0) {
         if (!workspace || workspace_bytes < pl.ws_bytes) return FLE_ERR_WORKSPACE;
         if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FLE_ERR_ALIGN;

@@ -218,20 +218,21 @@ __device__ __forceinline__ void atomic_max_f32(float* addr, float v) {
         atomicMin(reinterpret_cast<unsigned*>(addr), __float_as_uint(v));
 }
 
-__device__ __forceinline__ void load_bias32(const KParams& p, int64_t n0, float (&bv)[32]) {
-    if (p.bias == nullptr) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) bv[j] = 0.0f;
-    } else if (p.vec_bias && n0 + 32 <= p.N) {
+// v[j] += b[n0 + j] for the columns that exist, four at a time (no extra
+// 32-register copy of the bias).
+__device__ __forceinline__ void add_bias32(const KParams& p, int64_t n0, float (&v)[32]) {
+    if (p.bias == nullptr) return;
+    if (p.vec_bias && n0 + 32 <= p.N) {
         const float4* b4 = reinterpret_cast<const float4*>(p.bias + n0);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            float4 t = __ldg(b4 + j);
-            bv[4 * j] = t.x; bv[4 * j + 1] = t.y; bv[4 * j + 2] = t.z; bv[4 * j + 3] = t.w;
+        for (int i = 0; i < 8; ++i) {
+            const float4 t = __ldg(b4 + i);
+            v[4 * i] += t.x; v[4 * i + 1] += t.y; v[4 * i + 2] += t.z; v[4 * i + 3] += t.w;
         }
     } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) bv[j] = (n0 + j < p.N) ? __ldg(p.bias + n0 + j) : 0.0f;
+        for (int j = 0; j < 32; ++j)
+            if (n0 + j < p.N) v[j] += __ldg(p.bias + n0 + j);
     }
 }
 
@@ -249,10 +250,9 @@ struct EpiOut {
 template <int KIND>
 __device__ __forceinline__ void epi_store_direct(const KParams& p, const EpiOut& eo, int64_t m, int64_t n0,
                                                  float (&v)[32]) {
-    float bv[32];
-    load_bias32(p, n0, bv);
+    add_bias32(p, n0, v);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = epi_apply<KIND>(v[j] + bv[j], p);
+    for (int j = 0; j < 32; ++j) v[j] = epi_apply<KIND>(v[j], p);
     if (eo.tmap != nullptr) {
         // Row r of the block goes to staging row r; its eight 16-byte pieces
         // are placed at piece index (i ^ (r % 8)), the 128-byte swizzle the
@@ -288,14 +288,13 @@ __device__ __forceinline__ void epi_store_direct(const KParams& p, const EpiOut&
 // Direct layout, pool kind: folds complete windows of this 32-column chunk
 // into the running row maximum.
 __device__ __forceinline__ void epi_pool_direct(const KParams& p, int64_t n0, float (&v)[32], float& best) {
-    float bv[32];
-    load_bias32(p, n0, bv);
+    add_bias32(p, n0, v);
     const int k = p.pool_k;
     const float inv_k = 1.0f / static_cast<float>(k);
     float acc = 0.0f;
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
-        acc += v[j] + bv[j];
+        acc += v[j];
         if (((j + 1) & (k - 1)) == 0) {
             if (n0 + j + 1 <= p.pool_limit) {
                 float g = p.scale * gelu_erf(acc * inv_k);
@@ -527,22 +526,22 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         got = mbar_wait_bounded(bar_full(stage), phase, abort_flag, p.timeout_ns, kWhereConvFull);
                     got = __shfl_sync(0xffffffffu, got, 0);
                     if (!got) { ok = false; break; }
-                    // hi = x with the low 13 mantissa bits cleared (exactly a TF32
-                    // value); lo = x - hi (exact in fp32).  hi overwrites x in
-                    // place, lo goes to the same offset in the lo half.
-                    float4* hi4 = reinterpret_cast<float4*>(smem + stage * C::kStageBytes);
+                    // hi = x with the low 13 mantissa bits cleared (a TF32
+                    // value); lo = x - hi (exact in fp32) goes to the same
+                    // offset in the lo half.  The tensor core reads the raw x
+                    // of the hi half as exactly that hi: kind::tf32 truncates
+                    // an fp32 operand to TF32 (checked on the device by the
+                    // operand-conversion test).
+                    const float4* x4 = reinterpret_cast<const float4*>(smem + stage * C::kStageBytes);
                     float4* lo4 = reinterpret_cast<float4*>(smem + stage * C::kStageBytes + C::kLoadBytes);
                     constexpr int kVec = C::kLoadBytes / 16;
 #pragma unroll 4
                     for (int i = ct; i < kVec; i += 64) {
-                        float4 x = hi4[i];
-                        float4 h;
-                        h.x = __uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u);
-                        h.y = __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u);
-                        h.z = __uint_as_float(__float_as_uint(x.z) & 0xFFFFE000u);
-                        h.w = __uint_as_float(__float_as_uint(x.w) & 0xFFFFE000u);
-                        hi4[i] = h;
-                        lo4[i] = make_float4(x.x - h.x, x.y - h.y, x.z - h.z, x.w - h.w);
+                        const float4 x = x4[i];
+                        lo4[i] = make_float4(x.x - __uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u),
+                                             x.y - __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u),
+                                             x.z - __uint_as_float(__float_as_uint(x.z) & 0xFFFFE000u),
+                                             x.w - __uint_as_float(__float_as_uint(x.w) & 0xFFFFE000u));
                     }
                     fence_proxy_async_smem();
                     __syncwarp();

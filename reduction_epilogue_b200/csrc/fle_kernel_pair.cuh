@@ -10,29 +10,39 @@
 // 128 rows.
 //
 // Roles are those of fle_gemm_kernel.  Only the even ("leader") CTA's MMA
-// thread issues MMAs; both CTAs' producers load, and their copies are counted
-// on the leader's full barrier; the leader's commits are multicast to both
-// CTAs' empty and accumulator-full barriers; both CTAs' epilogues release the
-// leader's accumulator-empty barrier.  No load uses cluster multicast.
+// thread issues MMAs; the leader's commits are multicast to both CTAs' empty
+// and accumulator-full barriers; both CTAs' epilogues release the leader's
+// accumulator-empty barrier.  No load uses cluster multicast.
+//   TF32:   both CTAs' tile copies are counted on the leader's full barrier.
+//   3xTF32: each CTA's copies complete on its own full barrier; its split
+//           warps then write the TF32 low parts (x minus x with the low 13
+//           mantissa bits cleared; the tensor core reads the raw fp32 value
+//           as that truncated high part) and arrive on the leader's split
+//           barrier, which the MMA waits on.  The three products of each
+//           k-step accumulate in 128-deep slices of K, summed in registers
+//           (the tensor core's own accumulation rounds toward zero).
 #pragma once
 
 #include "fle_kernel.cuh"
 
 namespace fle {
 
-constexpr int kPairBN = 256;                      // pair tile N (B rows)
-constexpr int kPairBM = 256;                      // pair tile M (A rows)
+constexpr int kPairBN = 256;  // pair tile N (B rows)
+constexpr int kPairBM = 256;  // pair tile M (A rows)
 
+template <int PREC>
 struct PairCfg {
-    static constexpr int kABytes = kBM * kBK * 4;          // this CTA's 128 A rows
+    static constexpr int kABytes = kBM * kBK * 4;            // this CTA's 128 A rows
     static constexpr int kBBytes = (kPairBN / 2) * kBK * 4;  // this CTA's 128 B rows
-    static constexpr int kLoadBytes = kABytes + kBBytes;
+    static constexpr int kLoadBytes = kABytes + kBBytes;      // TMA bytes per stage and CTA
+    static constexpr int kStageBytes = kLoadBytes * (PREC == kPrec3xTF32 ? 2 : 1);
     static constexpr int kEpiStageBytes = kEpiWarps * kEpiTileBytes;  // TMA-store staging
-    static constexpr int kStages = (kSmemStageBudget - kEpiStageBytes) / kLoadBytes;  // 6
-    static constexpr int kTmemCols = 512;                    // 2 accumulator buffers x 256 columns
-    // full, empty per stage; accf, acce per buffer; drain; exit
-    static constexpr int kNumBars = 2 * kStages + 4 + 2;
-    static constexpr int kSmemBytes = 1024 + kStages * kLoadBytes + kEpiStageBytes + kNumBars * 8 + 32;
+    static constexpr int kStages = (kSmemStageBudget - kEpiStageBytes) / kStageBytes;
+    static constexpr int kTmemCols = 512;                     // 2 accumulator buffers x 256 columns
+    // full, split, empty per stage; accf, acce per buffer; drain; exit
+    static constexpr int kNumBars = 3 * kStages + 4 + 2;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kEpiStageBytes + kNumBars * 8 + 32;
+    static_assert(kStages >= 2, "need at least two stages");
     static_assert(kSmemBytes <= 232448, "exceeds 227 KB of shared memory per block");
 };
 
@@ -40,28 +50,31 @@ template <int PREC>
 __global__ void __launch_bounds__(kThreads, 1)
 fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmOut, const KParams p) {
-    static_assert(PREC == kPrecTF32, "CTA-pair kernel: single-pass TF32");
-    using C = PairCfg;
+    using C = PairCfg<PREC>;
+    constexpr bool k3x = (PREC == kPrec3xTF32);
     constexpr int S = C::kStages;
     constexpr uint32_t kIdesc = idesc_tf32(kPairBM, kPairBN);
+    constexpr int kChunkKb = k3x ? 4 : (1 << 30);  // k-blocks per TMEM accumulation chain
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    uint8_t* epi_stage = smem + S * C::kLoadBytes;
+    uint8_t* epi_stage = smem + S * C::kStageBytes;
     uint64_t* bars = reinterpret_cast<uint64_t*>(epi_stage + C::kEpiStageBytes);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
     auto bar_full = [&](int s) { return smem_u32(bars + s); };
-    auto bar_empty = [&](int s) { return smem_u32(bars + S + s); };
-    auto bar_accf = [&](int b) { return smem_u32(bars + 2 * S + b); };
-    auto bar_acce = [&](int b) { return smem_u32(bars + 2 * S + 2 + b); };
-    const uint32_t bar_drain = smem_u32(bars + 2 * S + 4);
-    const uint32_t bar_exit = smem_u32(bars + 2 * S + 5);
-    auto sA = [&](int s) { return sbase + s * C::kLoadBytes; };
-    auto sB = [&](int s) { return sbase + s * C::kLoadBytes + C::kABytes; };
+    auto bar_split = [&](int s) { return smem_u32(bars + S + s); };
+    auto bar_empty = [&](int s) { return smem_u32(bars + 2 * S + s); };
+    auto bar_accf = [&](int b) { return smem_u32(bars + 3 * S + b); };
+    auto bar_acce = [&](int b) { return smem_u32(bars + 3 * S + 2 + b); };
+    const uint32_t bar_drain = smem_u32(bars + 3 * S + 4);
+    const uint32_t bar_exit = smem_u32(bars + 3 * S + 5);
+    // stage s: [A | B | A lo | B lo]; the lo half exists for 3xTF32 only
+    auto sA = [&](int s) { return sbase + s * C::kStageBytes; };
+    auto sB = [&](int s) { return sbase + s * C::kStageBytes + C::kABytes; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -72,6 +85,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(bar_full(s), 1);
+            mbar_init(bar_split(s), 4);  // 2 split warps in each CTA of the pair
             mbar_init(bar_empty(s), 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -111,11 +125,20 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                         ok = false;
                         break;
                     }
-                    // The leader expects both CTAs' bytes on its own full barrier.
-                    if (rank == 0) mbar_arrive_expect_tx(bar_full(stage), 2 * C::kLoadBytes);
-                    const uint32_t leader_full = mapa_shared(bar_full(stage), 0);
-                    tma_load_2d_pair(sA(stage), &tmA, leader_full, kb * kBK, u.ta * kPairBM + rank * kBM);
-                    tma_load_2d_pair(sB(stage), &tmB, leader_full, kb * kBK, u.tb * kPairBN + rank * (kPairBN / 2));
+                    const int32_t ra = u.ta * kPairBM + static_cast<int32_t>(rank) * kBM;
+                    const int32_t rb = u.tb * kPairBN + static_cast<int32_t>(rank) * (kPairBN / 2);
+                    if constexpr (k3x) {
+                        // own barrier: this CTA's split warps wait for these bytes
+                        mbar_arrive_expect_tx(bar_full(stage), C::kLoadBytes);
+                        tma_load_2d(sA(stage), &tmA, bar_full(stage), kb * kBK, ra);
+                        tma_load_2d(sB(stage), &tmB, bar_full(stage), kb * kBK, rb);
+                    } else {
+                        // the leader expects both CTAs' bytes on its own full barrier
+                        if (rank == 0) mbar_arrive_expect_tx(bar_full(stage), 2 * C::kLoadBytes);
+                        const uint32_t leader_full = mapa_shared(bar_full(stage), 0);
+                        tma_load_2d_pair(sA(stage), &tmA, leader_full, kb * kBK, ra);
+                        tma_load_2d_pair(sB(stage), &tmB, leader_full, kb * kBK, rb);
+                    }
                     ++fills;
                     if (++stage == S) { stage = 0; phase ^= 1u; }
                 }
@@ -141,40 +164,88 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             sc.init(p, pair, num_pairs);
             Unit u;
             while (ok && sc.next(p, u)) {
-                if (!mbar_wait_bounded(bar_acce(buf), acc_phase ^ 1u, abort_flag, p.timeout_ns,
-                                       kWhereMmaAccEmpty)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after_sync();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kPairBN);
-                for (int kb = u.kb0; kb < u.kb1; ++kb) {
-                    if (!mbar_wait_bounded(bar_full(stage), phase, abort_flag, p.timeout_ns, kWhereMmaFull)) {
+                for (int kc = u.kb0; ok && kc < u.kb1; kc += kChunkKb) {
+                    const int kce = (u.kb1 - kc > kChunkKb) ? kc + kChunkKb : u.kb1;
+                    if (!mbar_wait_bounded(bar_acce(buf), acc_phase ^ 1u, abort_flag, p.timeout_ns,
+                                           kWhereMmaAccEmpty)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint64_t a_desc = smem_desc_sw128(sA(stage));
-                    const uint64_t b_desc = smem_desc_sw128(sB(stage));
+                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kPairBN);
+                    for (int kb = kc; kb < kce; ++kb) {
+                        const uint32_t wbar = k3x ? bar_split(stage) : bar_full(stage);
+                        if (!mbar_wait_bounded(wbar, phase, abort_flag, p.timeout_ns, kWhereMmaFull)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after_sync();
+                        const uint64_t a_hi = smem_desc_sw128(sA(stage));
+                        const uint64_t b_hi = smem_desc_sw128(sB(stage));
 #pragma unroll
-                    for (int k = 0; k < kBK / kUmmaK; ++k) {
-                        const uint64_t koff = static_cast<uint64_t>(k * 2);
-                        mma_tf32_pair(d_tmem, a_desc + koff, b_desc + koff, kIdesc, (kb > u.kb0 || k > 0) ? 1u : 0u);
+                        for (int k = 0; k < kBK / kUmmaK; ++k) {
+                            const uint64_t koff = static_cast<uint64_t>(k * 2);
+                            const uint32_t acc = (kb > kc || k > 0) ? 1u : 0u;
+                            if constexpr (k3x) {
+                                const uint64_t a_lo = smem_desc_sw128(sA(stage) + C::kLoadBytes);
+                                const uint64_t b_lo = smem_desc_sw128(sB(stage) + C::kLoadBytes);
+                                mma_tf32_pair(d_tmem, a_lo + koff, b_hi + koff, kIdesc, acc);
+                                mma_tf32_pair(d_tmem, a_hi + koff, b_lo + koff, kIdesc, 1u);
+                                mma_tf32_pair(d_tmem, a_hi + koff, b_hi + koff, kIdesc, 1u);
+                            } else {
+                                mma_tf32_pair(d_tmem, a_hi + koff, b_hi + koff, kIdesc, acc);
+                            }
+                        }
+                        mma_commit_pair_multicast(bar_empty(stage), 0x3);
+                        if (++stage == S) { stage = 0; phase ^= 1u; }
                     }
-                    mma_commit_pair_multicast(bar_empty(stage), 0x3);
-                    if (++stage == S) { stage = 0; phase ^= 1u; }
+                    if (!ok) break;
+                    mma_commit_pair_multicast(bar_accf(buf), 0x3);
+                    buf ^= 1;
+                    if (buf == 0) acc_phase ^= 1u;
                 }
-                if (!ok) break;
-                mma_commit_pair_multicast(bar_accf(buf), 0x3);
-                buf ^= 1;
-                if (buf == 0) acc_phase ^= 1u;
             }
             mma_commit_pair(bar_drain);
             volatile int never = 0;
             mbar_wait_bounded(bar_drain, 0, &never, p.timeout_ns, kWhereDrain);
         }
         __syncwarp();
-    } else if (warp >= 4) {
+    } else if (warp < 4) {
+        // ------------------------------------------------------------ 3xTF32 split (both CTAs)
+        if constexpr (k3x) {
+            const int ct = threadIdx.x - 64;  // 0..63
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            Sched sc;
+            sc.init(p, pair, num_pairs);
+            Unit u;
+            while (ok && sc.next(p, u)) {
+                for (int kb = u.kb0; kb < u.kb1; ++kb) {
+                    int got = 0;
+                    if (lane == 0)
+                        got = mbar_wait_bounded(bar_full(stage), phase, abort_flag, p.timeout_ns, kWhereConvFull);
+                    got = __shfl_sync(0xffffffffu, got, 0);
+                    if (!got) { ok = false; break; }
+                    const float4* x4 = reinterpret_cast<const float4*>(smem + stage * C::kStageBytes);
+                    float4* lo4 = reinterpret_cast<float4*>(smem + stage * C::kStageBytes + C::kLoadBytes);
+                    constexpr int kVec = C::kLoadBytes / 16;
+#pragma unroll 4
+                    for (int i = ct; i < kVec; i += 64) {
+                        const float4 x = x4[i];
+                        lo4[i] = make_float4(x.x - __uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u),
+                                             x.y - __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u),
+                                             x.z - __uint_as_float(__float_as_uint(x.z) & 0xFFFFE000u),
+                                             x.w - __uint_as_float(__float_as_uint(x.w) & 0xFFFFE000u));
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(mapa_shared(bar_split(stage), 0));
+                    if (++stage == S) { stage = 0; phase ^= 1u; }
+                }
+            }
+        }
+    } else {
         // ------------------------------------------------------------ epilogue (both CTAs)
         // Eight warps: lane quadrant warp % 4, half of the columns each.
         const int q = warp & 3;
@@ -188,17 +259,12 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         eo.stage_u32 = smem_u32(eo.stage);
         int buf = 0;
         uint32_t acc_phase = 0;
+        float accr[k3x ? kHalf * 32 : 1];  // 3xTF32: this thread's sums of the K slices
         Sched sc;
         sc.init(p, pair, num_pairs);
         Unit u;
-        while (sc.next(p, u)) {
-            int got = 0;
-            if (lane == 0)
-                got = mbar_wait_bounded(bar_accf(buf), acc_phase, abort_flag, p.timeout_ns, kWhereEpiAccFull);
-            got = __shfl_sync(0xffffffffu, got, 0);
-            if (!got) break;
-            tc_fence_after_sync();
-            const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * kPairBN);
+        bool ok = true;
+        while (ok && sc.next(p, u)) {
             const int64_t cols_left = p.N - static_cast<int64_t>(u.tb) * kPairBN;
             const int nchunks = static_cast<int>(cols_left >= kPairBN ? kPairBN / 32 : (cols_left + 31) / 32);
             const int mine = nchunks - c_lo < 0 ? 0 : (nchunks - c_lo > kHalf ? kHalf : nchunks - c_lo);
@@ -206,6 +272,14 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             Unit uh = u;
             uh.ta = 2 * u.ta + static_cast<int>(rank);
             eo.row0 = static_cast<int64_t>(uh.ta) * kBM + q * 32;
+            auto wait_acc = [&]() -> bool {
+                int got = 0;
+                if (lane == 0)
+                    got = mbar_wait_bounded(bar_accf(buf), acc_phase, abort_flag, p.timeout_ns, kWhereEpiAccFull);
+                got = __shfl_sync(0xffffffffu, got, 0);
+                if (got) tc_fence_after_sync();
+                return got != 0;
+            };
             auto release_acc = [&]() {
                 tc_fence_before_sync();
                 __syncwarp();
@@ -213,29 +287,81 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 buf ^= 1;
                 if (buf == 0) acc_phase ^= 1u;
             };
+            auto t_row = [&]() {
+                return tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * kPairBN);
+            };
+
+            uint32_t t_acc = 0;
+            if constexpr (k3x) {
+#pragma unroll
+                for (int j = 0; j < kHalf * 32; ++j) accr[j] = 0.0f;
+                for (int kc = u.kb0; kc < u.kb1; kc += kChunkKb) {
+                    if (!wait_acc()) { ok = false; break; }
+                    const uint32_t tr = t_row();
+#pragma unroll
+                    for (int lc = 0; lc < kHalf; ++lc) {
+                        if (lc >= mine) break;
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            float v[16];
+                            tmem_ld16_wait(tr + (c_lo + lc) * 32 + h * 16, v);
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) accr[lc * 32 + h * 16 + j] += v[j];
+                        }
+                    }
+                    release_acc();
+                }
+                if (!ok) break;
+            } else {
+                if (!wait_acc()) break;
+                t_acc = t_row();
+            }
 
             if (!u.partial) {
                 float best = -INFINITY;
+                if constexpr (k3x) {
+#pragma unroll
+                    for (int lc = 0; lc < kHalf; ++lc) {
+                        if (lc < mine) {
+                            float v[32];
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] = accr[lc * 32 + j];
+                            epi_chunk<false, kPairBN>(p, uh, r, c_lo + lc, v, best, eo);
+                        }
+                    }
+                } else {
 #pragma unroll 1
-                for (int lc = 0; lc < mine; ++lc) {
-                    float v[32];
-                    tmem_ld32_wait(t_acc + (c_lo + lc) * 32, v);
-                    epi_chunk<false, kPairBN>(p, uh, r, c_lo + lc, v, best, eo);
+                    for (int lc = 0; lc < mine; ++lc) {
+                        float v[32];
+                        tmem_ld32_wait(t_acc + (c_lo + lc) * 32, v);
+                        epi_chunk<false, kPairBN>(p, uh, r, c_lo + lc, v, best, eo);
+                    }
                 }
                 epi_finish<false>(p, uh, r, best);
-                release_acc();
+                if constexpr (!k3x) release_acc();
             } else {
                 // column-major partial tile: element (row, col) at col * 128 + row
                 float* slot = p.ws + static_cast<size_t>(2 * blockIdx.x + u.slot) * kBM * kPairBN;
-#pragma unroll 1
-                for (int lc = 0; lc < mine; ++lc) {
-                    float v[32];
-                    tmem_ld32_wait(t_acc + (c_lo + lc) * 32, v);
-                    float* d = slot + static_cast<size_t>((c_lo + lc) * 32) * kBM + r;
+                if constexpr (k3x) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) __stcg(d + j * kBM, v[j]);
+                    for (int lc = 0; lc < kHalf; ++lc) {
+                        if (lc < mine) {
+                            float* d = slot + static_cast<size_t>((c_lo + lc) * 32) * kBM + r;
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) __stcg(d + j * kBM, accr[lc * 32 + j]);
+                        }
+                    }
+                } else {
+#pragma unroll 1
+                    for (int lc = 0; lc < mine; ++lc) {
+                        float v[32];
+                        tmem_ld32_wait(t_acc + (c_lo + lc) * 32, v);
+                        float* d = slot + static_cast<size_t>((c_lo + lc) * 32) * kBM + r;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) __stcg(d + j * kBM, v[j]);
+                    }
+                    release_acc();
                 }
-                release_acc();
                 const int64_t tsk = u.sk_tile;
                 const int first = sk_cta_of(tsk * p.num_kb, p.sk_iters, p.sk_grid);
                 const int last = sk_cta_of((tsk + 1) * p.num_kb - 1, p.sk_iters, p.sk_grid);

@@ -229,19 +229,21 @@ def test_plan_choices(fle):
     assert "swap=0" in fle.plan_string(2048, 8192, 8192, d)
 
 
-def test_tf32_input_conversion_probe(fle, capsys):
-    # Records how the tensor core reads an fp32 operand in kind::tf32 (the low
-    # 13 mantissa bits dropped, or rounded).  Informational; the 3xTF32 split
-    # masks the high part explicitly, so it depends on neither behaviour.
+def test_tf32_input_conversion_truncates(fle, capsys):
+    # The 3xTF32 split writes only the low part lo = x - trunc13(x) and lets
+    # the tensor core read the raw fp32 x as the high part, which is exact
+    # only if kind::tf32 drops the low 13 mantissa bits of an fp32 operand
+    # (rather than rounding).  Checked here on values whose dropped bits
+    # would round up.
     v = 1.0 + 2.0 ** -11 + 2.0 ** -12
     x = torch.full((1, 4), v, device="cuda")
     W = torch.ones(1, 4, device="cuda")
     out = _run(fle, x, W, None, "none", "tf32")
     got = float(out[0, 0])
     trunc, rn = 4.0, 4.0 * (1.0 + 2.0 ** -10)
-    assert got in (trunc, rn), got
     with capsys.disabled():
-        print(f"\n[tf32 operand conversion: {'truncate' if got == trunc else 'round-to-nearest'}]")
+        print(f"\n[tf32 operand conversion: {'truncate' if got == trunc else 'round-to-nearest' if got == rn else got}]")
+    assert got == trunc, got
 
 
 def test_tensor_core_accumulation_rounding_probe(fle, capsys):

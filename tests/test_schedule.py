@@ -113,9 +113,9 @@ def test_headline_shape_splits_only_the_last_wave():
     halves = [r for rows in per_cta for r in rows if r[5]]
     assert len(halves) == 68
     assert {(int(r[3]), int(r[4])) for r in halves} == {(0, 128), (128, 256)}
-    # 3xTF32 keeps single-CTA 128x128 tiles: 16 x 64 = 1024 tiles
+    # 3xTF32 runs the same 256x256 pair tiles (and the same schedule)
     grid3, per3 = collect(2048, 8192, 8192, fle.desc_for("scale_hardtanh_gelu", "3xtf32"), 148)
-    assert grid3 == 148 and sum(len(r) for r in per3) == 1024
+    assert grid3 == 74 and sum(int(r[4]) - int(r[3]) for rows in per3 for r in rows) == 256 * 256
 
 
 def test_weight_streamed_once_shapes_use_every_sm():
