@@ -96,6 +96,23 @@ def profiled_traffic(workload: str, precision: str):
         return None
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time: every rank contributes its own, all receive
+    the maximum (the job is as fast as its slowest replica)."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput_tflops(flops_per_step: float, world: int, steps: int, total_ms: float) -> float:
+    """Whole-job throughput: the work of all ranks' steps over the slowest
+    rank's time (weak scaling: each rank runs its own replica)."""
+    return flops_per_step * world * steps / (total_ms * 1e-3) / 1e12
+
+
 def algorithmic(M, K, N, problem, variant=None):
     """(flops, bytes, output elements) one call must do.  The pooled-weight
     variants do the GEMM at N/16 columns; per call they also read W once and
@@ -310,12 +327,9 @@ def run_fle(args, name, dist_ctx):
     total_ms = sum(step_ms)
     if fle.device_status(stream) != 0:
         raise RuntimeError("device status set during the timed steps")
-    t_max = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t_max, op=torch.distributed.ReduceOp.MAX)
-    total_ms = float(t_max.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / args.steps
-    value = flops * world * args.steps / (total_ms * 1e-3) / 1e12
+    value = job_throughput_tflops(flops, world, args.steps, total_ms)
 
     # end to end through the public call: pinned host inputs in, result out
     e2e = None
@@ -349,10 +363,8 @@ def run_fle(args, name, dist_ctx):
             outh.copy_(out, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            torch.distributed.all_reduce(e_ms, op=torch.distributed.ReduceOp.MAX)
-        e2e = {"value": flops * world * e2e_steps / (float(e_ms.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": job_throughput_tflops(flops, world, e2e_steps, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": (4 * (M * K + N * K + N) if copy_w else 4 * M * K),
                "d2h_bytes_per_step": 4 * out_elems, "steps": e2e_steps}
 
