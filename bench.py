@@ -380,6 +380,9 @@ def run_fle(args, name, dist_ctx):
         roof = {"bound": "tensor", "achieved": achieved, "peak": tf32_peak, "unit": "TFLOP/s",
                 "frac": achieved / tf32_peak,
                 "peak_source": f"{peak_src} bf16 {peaks['bf16_tflops']} TFLOP/s x 1.1/2.25 (TF32:BF16 nominal)"}
+        if args.precision == "3xtf32":
+            # the tensor core executes three TF32 products per term
+            roof["frac_of_3pass"] = 3 * achieved / tf32_peak
     else:
         achieved = nbytes / avg_launch_s / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",

@@ -144,6 +144,7 @@ int check_shape(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d) {
 struct Plan {
     bool swap = false;
     bool pair = false;         // 256x256 tiles on CTA pairs (cta_group::2)
+    int bk = 32;               // k-block width in fp32
     int bn = 256;
     int prec = fle::kPrecTF32;
     int stages = 0;
@@ -203,7 +204,8 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
     pl.tiles_a = static_cast<int>((Ma + tile_m - 1) / tile_m);
     pl.tiles_b = static_cast<int>((Nb + pl.bn - 1) / pl.bn);
     pl.tiles = pl.tiles_a * pl.tiles_b;
-    pl.num_kb = static_cast<int>((K + fle::kBK - 1) / fle::kBK);
+    pl.bk = fle::kBK;
+    pl.num_kb = static_cast<int>((K + pl.bk - 1) / pl.bk);
     pl.stages = pl.pair ? (pl.prec == fle::kPrec3xTF32 ? fle::PairCfg<fle::kPrec3xTF32>::kStages
                                                        : fle::PairCfg<fle::kPrecTF32>::kStages)
                         : stages_for(pl.bn, pl.prec);
@@ -217,13 +219,15 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
     const bool w_shared = (pl.swap ? pl.tiles_b : pl.tiles_a) > 1;
     const char* ov = sched_override();
     const bool force_dp = std::strcmp(ov, "dp") == 0;
+    // the stream-K minimum is 16 k-blocks of 32 (512 of K) per CTA
+    const int64_t min_iters = kMinSkIters * fle::kBK / pl.bk;
     pl.dp_tiles = static_cast<int>(T);
     pl.grid = static_cast<int>(T < G ? T : G);
     pl.sk_grid = 0;
-    if (!force_dp && T % G != 0 && pl.num_kb >= 2 * kMinSkIters) {
+    if (!force_dp && T % G != 0 && pl.num_kb >= 2 * min_iters) {
         if (!w_shared && T < G) {
             // every weight tile is read by one unit: spread all k-blocks over the SMs
-            const int64_t g_sk = std::min<int64_t>(G, iters / kMinSkIters);
+            const int64_t g_sk = std::min<int64_t>(G, iters / min_iters);
             if (g_sk > T) {
                 pl.dp_tiles = 0;
                 pl.grid = static_cast<int>(g_sk);
@@ -233,7 +237,7 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
             // full waves data-parallel; the R tiles of the last partial wave
             // split into S k-aligned parts on R*S CTAs
             const int64_t R = T % G;
-            const int64_t S = std::min<int64_t>(G / R, pl.num_kb / kMinSkIters);
+            const int64_t S = std::min<int64_t>(G / R, pl.num_kb / min_iters);
             if (S >= 2) {
                 pl.dp_tiles = static_cast<int>(T - R);
                 pl.grid = static_cast<int>(T > G ? G : R * S);
@@ -347,10 +351,10 @@ bool sync_check_enabled() {
 int plan_to_string(const Plan& pl, char* buf, size_t n) {
     if (!buf || n == 0) return FLE_ERR_NULL;
     std::snprintf(buf, n,
-                  "tile=%dx%d pair=%d swap=%d prec=%s stages=%d tiles=%dx%d kblocks=%d dp_tiles=%d sk_tiles=%d "
+                  "tile=%dx%d pair=%d swap=%d prec=%s stages=%d bk=%d tiles=%dx%d kblocks=%d dp_tiles=%d sk_tiles=%d "
                   "sk_kblocks=%lld sk_grid=%d grid=%d workspace=%zu",
                   pl.pair ? fle::kPairBM : fle::kBM, pl.bn, pl.pair ? 1 : 0, pl.swap ? 1 : 0,
-                  pl.prec == fle::kPrecTF32 ? "tf32" : "3xtf32", pl.stages,
+                  pl.prec == fle::kPrecTF32 ? "tf32" : "3xtf32", pl.stages, pl.bk,
                   pl.tiles_a, pl.tiles_b, pl.num_kb, pl.dp_tiles, pl.sk_tiles, (long long)pl.sk_iters, pl.sk_grid, pl.grid,
                   pl.ws_bytes);
     return FLE_OK;

@@ -32,8 +32,9 @@ constexpr int kPairBM = 256;  // pair tile M (A rows)
 
 template <int PREC>
 struct PairCfg {
-    static constexpr int kABytes = kBM * kBK * 4;            // this CTA's 128 A rows
-    static constexpr int kBBytes = (kPairBN / 2) * kBK * 4;  // this CTA's 128 B rows
+    static constexpr int kBKW = kBK;  // k-block width: 32 fp32, one 128-byte swizzle row
+    static constexpr int kABytes = kBM * kBKW * 4;            // this CTA's 128 A rows
+    static constexpr int kBBytes = (kPairBN / 2) * kBKW * 4;  // this CTA's 128 B rows
     static constexpr int kLoadBytes = kABytes + kBBytes;      // TMA bytes per stage and CTA
     static constexpr int kStageBytes = kLoadBytes * (PREC == kPrec3xTF32 ? 2 : 1);
     static constexpr int kEpiStageBytes = kEpiWarps * kEpiTileBytes;  // TMA-store staging
@@ -54,7 +55,8 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     constexpr bool k3x = (PREC == kPrec3xTF32);
     constexpr int S = C::kStages;
     constexpr uint32_t kIdesc = idesc_tf32(kPairBM, kPairBN);
-    constexpr int kChunkKb = k3x ? 4 : (1 << 30);  // k-blocks per TMEM accumulation chain
+    constexpr int kBKW = C::kBKW;
+    constexpr int kChunkKb = k3x ? 128 / kBKW : (1 << 30);  // k-blocks per TMEM accumulation chain
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -130,14 +132,14 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     if constexpr (k3x) {
                         // own barrier: this CTA's split warps wait for these bytes
                         mbar_arrive_expect_tx(bar_full(stage), C::kLoadBytes);
-                        tma_load_2d(sA(stage), &tmA, bar_full(stage), kb * kBK, ra);
-                        tma_load_2d(sB(stage), &tmB, bar_full(stage), kb * kBK, rb);
+                        tma_load_2d(sA(stage), &tmA, bar_full(stage), kb * kBKW, ra);
+                        tma_load_2d(sB(stage), &tmB, bar_full(stage), kb * kBKW, rb);
                     } else {
                         // the leader expects both CTAs' bytes on its own full barrier
                         if (rank == 0) mbar_arrive_expect_tx(bar_full(stage), 2 * C::kLoadBytes);
                         const uint32_t leader_full = mapa_shared(bar_full(stage), 0);
-                        tma_load_2d_pair(sA(stage), &tmA, leader_full, kb * kBK, ra);
-                        tma_load_2d_pair(sB(stage), &tmB, leader_full, kb * kBK, rb);
+                        tma_load_2d_pair(sA(stage), &tmA, leader_full, kb * kBKW, ra);
+                        tma_load_2d_pair(sB(stage), &tmB, leader_full, kb * kBKW, rb);
                     }
                     ++fills;
                     if (++stage == S) { stage = 0; phase ^= 1u; }
@@ -180,15 +182,17 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                             break;
                         }
                         tc_fence_after_sync();
-                        const uint64_t a_hi = smem_desc_sw128(sA(stage));
-                        const uint64_t b_hi = smem_desc_sw128(sB(stage));
+                        auto desc = [](uint32_t a) { return smem_desc_sw128(a); };
+                        const uint64_t a_hi = desc(sA(stage));
+                        const uint64_t b_hi = desc(sB(stage));
 #pragma unroll
-                        for (int k = 0; k < kBK / kUmmaK; ++k) {
+                        for (int k = 0; k < kBKW / kUmmaK; ++k) {
+                            // advance 8 fp32 = 32 bytes along K inside the swizzle atom
                             const uint64_t koff = static_cast<uint64_t>(k * 2);
                             const uint32_t acc = (kb > kc || k > 0) ? 1u : 0u;
                             if constexpr (k3x) {
-                                const uint64_t a_lo = smem_desc_sw128(sA(stage) + C::kLoadBytes);
-                                const uint64_t b_lo = smem_desc_sw128(sB(stage) + C::kLoadBytes);
+                                const uint64_t a_lo = desc(sA(stage) + C::kLoadBytes);
+                                const uint64_t b_lo = desc(sB(stage) + C::kLoadBytes);
                                 mma_tf32_pair(d_tmem, a_lo + koff, b_hi + koff, kIdesc, acc);
                                 mma_tf32_pair(d_tmem, a_hi + koff, b_lo + koff, kIdesc, 1u);
                                 mma_tf32_pair(d_tmem, a_hi + koff, b_hi + koff, kIdesc, 1u);

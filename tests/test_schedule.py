@@ -52,7 +52,9 @@ def test_schedule_covers_every_kblock_once(M, K, N, problem, precision, sms):
     desc = fle.desc_for(problem, precision)
     grid, per_cta = collect(M, K, N, desc, sms)
     assert 1 <= grid <= sms
-    num_kb = math.ceil(K / 32)
+    # k-blocks are 32 wide, or 16 wide for 3xTF32 on CTA pairs
+    num_kb = max(int(r[4]) for rows in per_cta for r in rows)
+    assert num_kb == math.ceil(K / 32) or (precision == "3xtf32" and num_kb == math.ceil(K / 16))
     cover = defaultdict(list)  # tile -> [(kb0, kb1, cta, row)]
     for c, rows in enumerate(per_cta):
         partial_slots = []
