@@ -32,8 +32,8 @@ struct DeviceInfo {
 // Co-resident 2-CTA clusters of a pair kernel on the current device.
 template <int PREC>
 int max_active_pairs() {
-    auto kern = fle::fle_gemm_pair_kernel<PREC>;
-    const int smem = fle::PairCfg<PREC>::kSmemBytes;
+    auto kern = fle::fle_gemm_pair_kernel<PREC, 1, fle::kPairBN, false>;
+    const int smem = fle::PairCfg<PREC, 1>::kSmemBytes;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return 0;
     cudaLaunchConfig_t cfg = {};
@@ -144,6 +144,7 @@ int check_shape(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d) {
 struct Plan {
     bool swap = false;
     bool pair = false;         // 256x256 tiles on CTA pairs (cta_group::2)
+    int kps = 1;               // k-blocks per ring stage
     int bk = 32;               // k-block width in fp32
     int bn = 256;
     int prec = fle::kPrecTF32;
@@ -159,10 +160,18 @@ struct Plan {
     size_t ws_bytes = 0;       // ... then one arrival counter per stream-K tile
 };
 
-int stages_for(int bn, int prec) {
-    const int stage = (fle::kBM + bn) * fle::kBK * 4 * (prec == fle::kPrec3xTF32 ? 2 : 1);
-    const int s = fle::kSmemStageBudget / stage;
+// Ring depth of the single-CTA kernel (mirrors Cfg::kStages).
+int stages_for(int bn, int prec, int kps, bool swap) {
+    const int stage = kps * (fle::kBM + bn) * fle::kBK * 4 * (prec == fle::kPrec3xTF32 ? 2 : 1);
+    const int s = (fle::kSmemStageBudget - (swap ? 0 : fle::kEpiWarps * fle::kEpiTileBytes)) / stage;
     return s > 8 ? 8 : s;
+}
+
+// Ring depth of the pair kernel (mirrors PairCfg::kStages).
+int pair_stages_for(int bn, int prec, int kps, bool swap) {
+    const int stage = kps * (fle::kBM + bn / 2) * fle::kBK * 4 * (prec == fle::kPrec3xTF32 ? 2 : 1);
+    const int s = (fle::kSmemStageBudget - (swap ? 0 : fle::kEpiWarps * fle::kEpiTileBytes)) / stage;
+    return s > 12 ? 12 : s;
 }
 
 // Fewest k-blocks (of 32) a CTA takes in the stream-K part of a schedule.
@@ -172,6 +181,16 @@ const char* sched_override() {
     static const char* v = [] {
         const char* e = std::getenv("FLE_SCHED");
         return e ? e : "";
+    }();
+    return v;
+}
+
+// k-blocks per ring stage: FLE_KPS=1 or 2 overrides the planner's choice
+// (single-pass TF32 only; 3xTF32 stages hold one k-block).
+int kps_override() {
+    static int v = [] {
+        const char* e = std::getenv("FLE_KPS");
+        return (e && (e[0] == '1' || e[0] == '2')) ? e[0] - '0' : 0;
     }();
     return v;
 }
@@ -189,13 +208,21 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
     Plan pl;
     pl.prec = (d->precision == FLE_PREC_3XTF32) ? fle::kPrec3xTF32 : fle::kPrecTF32;
     pl.swap = (M <= 128) && d->kind != FLE_EPI_AVGPOOL_GELU_SCALE_ROWMAX;
-    pl.pair = !pl.swap && M > 128 && pairs > 0 && !pair_disabled();
-    int tile_m = fle::kBM;
-    if (pl.pair) {
-        tile_m = fle::kPairBM;
-        pl.bn = fle::kPairBN;
-    } else if (pl.swap) {
+    // CTA pairs: 256 A rows per tile, each CTA loading half of the B rows.
+    // Swapped (skinny) shapes use them in TF32 when the weight has at least
+    // a full wave of 256-row tiles (measured: the pair kernel then streams
+    // the weight faster; with fewer tiles, or in 3xTF32, the one-CTA kernel
+    // is faster).
+    const bool pairs_ok = pairs > 0 && !pair_disabled();
+    if (pl.swap)
+        pl.pair = pairs_ok && pl.prec == fle::kPrecTF32 && (N + fle::kPairBM - 1) / fle::kPairBM >= pairs;
+    else
+        pl.pair = pairs_ok && M > 128;
+    int tile_m = pl.pair ? fle::kPairBM : fle::kBM;
+    if (pl.swap) {
         pl.bn = M <= 32 ? 32 : (M <= 64 ? 64 : 128);
+    } else if (pl.pair) {
+        pl.bn = fle::kPairBN;
     } else {
         pl.bn = (pl.prec == fle::kPrec3xTF32) ? 128 : 256;
     }
@@ -206,29 +233,36 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
     pl.tiles = pl.tiles_a * pl.tiles_b;
     pl.bk = fle::kBK;
     pl.num_kb = static_cast<int>((K + pl.bk - 1) / pl.bk);
-    pl.stages = pl.pair ? (pl.prec == fle::kPrec3xTF32 ? fle::PairCfg<fle::kPrec3xTF32>::kStages
-                                                       : fle::PairCfg<fle::kPrecTF32>::kStages)
-                        : stages_for(pl.bn, pl.prec);
+    // Two k-blocks per ring stage (TF32): measured faster on the swapped
+    // skinny kernel and on pair plans of two or more full waves; plans with
+    // fewer tiles keep the deeper one-k-block ring.
+    pl.kps = 1;
+    if (pl.prec == fle::kPrecTF32) {
+        const int64_t tiles = static_cast<int64_t>(pl.tiles_a) * pl.tiles_b;
+        if (pl.swap || (pl.pair && tiles >= 2 * static_cast<int64_t>(pairs))) pl.kps = 2;
+        if (kps_override() != 0) pl.kps = kps_override();
+    }
+    pl.stages = pl.pair ? pair_stages_for(pl.bn, pl.prec, pl.kps, pl.swap) : stages_for(pl.bn, pl.prec, pl.kps, pl.swap);
 
     // The schedule runs over CTAs, or over CTA pairs in pair mode.
     const int64_t T = pl.tiles;
     const int64_t G = pl.pair ? pairs : sms;
     const int64_t iters = T * pl.num_kb;
-    // Is a weight tile used by more than one tile of the output?  Then CTAs
-    // sharing it must walk K in step to reuse it from L2.
-    const bool w_shared = (pl.swap ? pl.tiles_b : pl.tiles_a) > 1;
     const char* ov = sched_override();
     const bool force_dp = std::strcmp(ov, "dp") == 0;
+    const bool force_sk = std::strcmp(ov, "sk") == 0;
     // the stream-K minimum is 16 k-blocks of 32 (512 of K) per CTA
     const int64_t min_iters = kMinSkIters * fle::kBK / pl.bk;
     pl.dp_tiles = static_cast<int>(T);
     pl.grid = static_cast<int>(T < G ? T : G);
     pl.sk_grid = 0;
     if (!force_dp && T % G != 0 && pl.num_kb >= 2 * min_iters) {
-        if (!w_shared && T < G) {
-            // every weight tile is read by one unit: spread all k-blocks over the SMs
+        if (force_sk) {
+            // spread all k-blocks evenly over all SMs (measured no faster
+            // than the k-aligned split below on any of the benchmark shapes,
+            // and slower on some)
             const int64_t g_sk = std::min<int64_t>(G, iters / min_iters);
-            if (g_sk > T) {
+            if (g_sk > T || (T > G && g_sk >= 2)) {
                 pl.dp_tiles = 0;
                 pl.grid = static_cast<int>(g_sk);
                 pl.sk_grid = pl.grid;
@@ -258,11 +292,14 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
     return pl;
 }
 
-template <int BN, int PREC, bool SWAP>
+// after_prep: the previous kernel in the stream is this call's prep kernel,
+// which writes nothing the GEMM reads before griddep_wait(); the GEMM is then
+// launched with programmatic stream serialization and starts during it.
+template <int BN, int PREC, bool SWAP, int KPS>
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to, const KParams& p,
-                        int grid, cudaStream_t st) {
-    using C = fle::Cfg<BN, PREC, SWAP>;
-    auto kern = fle::fle_gemm_kernel<BN, PREC, SWAP>;
+                        int grid, bool after_prep, cudaStream_t st) {
+    using C = fle::Cfg<BN, PREC, SWAP, KPS>;
+    auto kern = fle::fle_gemm_kernel<BN, PREC, SWAP, KPS>;
     static bool attr_set[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -271,52 +308,96 @@ cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    kern<<<grid, fle::kThreads, C::kSmemBytes, st>>>(ta, tb, to, p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(fle::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = after_prep ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, to, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
-template <int PREC>
+template <int PREC, int KPS, int BN = fle::kPairBN, bool SWAP = false>
 cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to, const KParams& p,
-                             int pairs, cudaStream_t st) {
-    // max_active_pairs() set the kernel's shared-memory attribute when the
-    // device was probed.
+                             int pairs, bool after_prep, cudaStream_t st) {
+    using C = fle::PairCfg<PREC, KPS, BN, SWAP>;
+    auto kern = fle::fle_gemm_pair_kernel<PREC, KPS, BN, SWAP>;
+    static bool attr_set[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
     cfg.blockDim = dim3(fle::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = fle::PairCfg<PREC>::kSmemBytes;
+    cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, fle::fle_gemm_pair_kernel<PREC>, ta, tb, to, p);
+    cfg.numAttrs = after_prep ? 2 : 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, to, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
 cudaError_t dispatch(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
-                     const KParams& p, cudaStream_t st) {
-    const bool tf32 = pl.prec == fle::kPrecTF32;
-    if (pl.pair)
-        return tf32 ? launch_gemm_pair<fle::kPrecTF32>(ta, tb, to, p, pl.grid, st)
-                    : launch_gemm_pair<fle::kPrec3xTF32>(ta, tb, to, p, pl.grid, st);
+                     const KParams& p, bool after_prep, cudaStream_t st) {
+    using namespace fle;
+    const bool tf32 = pl.prec == kPrecTF32;
+    const bool two = pl.kps == 2;  // TF32 only
+    if (pl.pair && !pl.swap) {
+        if (!tf32) return launch_gemm_pair<kPrec3xTF32, 1>(ta, tb, to, p, pl.grid, after_prep, st);
+        return two ? launch_gemm_pair<kPrecTF32, 2>(ta, tb, to, p, pl.grid, after_prep, st)
+                   : launch_gemm_pair<kPrecTF32, 1>(ta, tb, to, p, pl.grid, after_prep, st);
+    }
+    if (pl.pair) {
+        switch (pl.bn) {
+#define FLE_PAIR_SWAP_CASE(bn)                                                                             \
+    case bn:                                                                                               \
+        if (!tf32) return launch_gemm_pair<kPrec3xTF32, 1, bn, true>(ta, tb, to, p, pl.grid, after_prep, st); \
+        return two ? launch_gemm_pair<kPrecTF32, 2, bn, true>(ta, tb, to, p, pl.grid, after_prep, st)      \
+                   : launch_gemm_pair<kPrecTF32, 1, bn, true>(ta, tb, to, p, pl.grid, after_prep, st);
+            FLE_PAIR_SWAP_CASE(32)
+            FLE_PAIR_SWAP_CASE(64)
+            FLE_PAIR_SWAP_CASE(128)
+#undef FLE_PAIR_SWAP_CASE
+            default: return cudaErrorInvalidConfiguration;
+        }
+    }
     if (!pl.swap) {
-        if (tf32 && pl.bn == 256) return launch_gemm<256, fle::kPrecTF32, false>(ta, tb, to, p, pl.grid, st);
-        if (!tf32 && pl.bn == 128) return launch_gemm<128, fle::kPrec3xTF32, false>(ta, tb, to, p, pl.grid, st);
+        if (tf32 && pl.bn == 256)
+            return two ? launch_gemm<256, kPrecTF32, false, 2>(ta, tb, to, p, pl.grid, after_prep, st)
+                       : launch_gemm<256, kPrecTF32, false, 1>(ta, tb, to, p, pl.grid, after_prep, st);
+        if (!tf32 && pl.bn == 128) return launch_gemm<128, kPrec3xTF32, false, 1>(ta, tb, to, p, pl.grid, after_prep, st);
     } else {
         switch (pl.bn) {
             case 32:
-                return tf32 ? launch_gemm<32, fle::kPrecTF32, true>(ta, tb, to, p, pl.grid, st)
-                            : launch_gemm<32, fle::kPrec3xTF32, true>(ta, tb, to, p, pl.grid, st);
+                if (!tf32) return launch_gemm<32, kPrec3xTF32, true, 1>(ta, tb, to, p, pl.grid, after_prep, st);
+                return two ? launch_gemm<32, kPrecTF32, true, 2>(ta, tb, to, p, pl.grid, after_prep, st)
+                           : launch_gemm<32, kPrecTF32, true, 1>(ta, tb, to, p, pl.grid, after_prep, st);
             case 64:
-                return tf32 ? launch_gemm<64, fle::kPrecTF32, true>(ta, tb, to, p, pl.grid, st)
-                            : launch_gemm<64, fle::kPrec3xTF32, true>(ta, tb, to, p, pl.grid, st);
+                if (!tf32) return launch_gemm<64, kPrec3xTF32, true, 1>(ta, tb, to, p, pl.grid, after_prep, st);
+                return two ? launch_gemm<64, kPrecTF32, true, 2>(ta, tb, to, p, pl.grid, after_prep, st)
+                           : launch_gemm<64, kPrecTF32, true, 1>(ta, tb, to, p, pl.grid, after_prep, st);
             case 128:
-                return tf32 ? launch_gemm<128, fle::kPrecTF32, true>(ta, tb, to, p, pl.grid, st)
-                            : launch_gemm<128, fle::kPrec3xTF32, true>(ta, tb, to, p, pl.grid, st);
+                if (!tf32) return launch_gemm<128, kPrec3xTF32, true, 1>(ta, tb, to, p, pl.grid, after_prep, st);
+                return two ? launch_gemm<128, kPrecTF32, true, 2>(ta, tb, to, p, pl.grid, after_prep, st)
+                           : launch_gemm<128, kPrecTF32, true, 1>(ta, tb, to, p, pl.grid, after_prep, st);
             default: break;
         }
     }
@@ -351,10 +432,10 @@ bool sync_check_enabled() {
 int plan_to_string(const Plan& pl, char* buf, size_t n) {
     if (!buf || n == 0) return FLE_ERR_NULL;
     std::snprintf(buf, n,
-                  "tile=%dx%d pair=%d swap=%d prec=%s stages=%d bk=%d tiles=%dx%d kblocks=%d dp_tiles=%d sk_tiles=%d "
+                  "tile=%dx%d pair=%d swap=%d prec=%s stages=%d kps=%d tiles=%dx%d kblocks=%d dp_tiles=%d sk_tiles=%d "
                   "sk_kblocks=%lld sk_grid=%d grid=%d workspace=%zu",
                   pl.pair ? fle::kPairBM : fle::kBM, pl.bn, pl.pair ? 1 : 0, pl.swap ? 1 : 0,
-                  pl.prec == fle::kPrecTF32 ? "tf32" : "3xtf32", pl.stages, pl.bk,
+                  pl.prec == fle::kPrecTF32 ? "tf32" : "3xtf32", pl.stages, pl.kps,
                   pl.tiles_a, pl.tiles_b, pl.num_kb, pl.dp_tiles, pl.sk_tiles, (long long)pl.sk_iters, pl.sk_grid, pl.grid,
                   pl.ws_bytes);
     return FLE_OK;
@@ -477,7 +558,7 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
     const float* B = pl.swap ? x : W;
     st = encode_operand(&ta, A, p.Ma, K, fle::kBM);
     if (st != FLE_OK) return st;
-    st = encode_operand(&tb, B, p.Nb, K, pl.pair ? fle::kPairBN / 2 : pl.bn);
+    st = encode_operand(&tb, B, p.Nb, K, pl.pair ? pl.bn / 2 : pl.bn);
     if (st != FLE_OK) return st;
 
     if (log_enabled()) {
@@ -487,7 +568,8 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
                      (long long)N, d->kind, line);
     }
 
-    if (pool || pl.sk_tiles > 0) {
+    const bool prep = pool || pl.sk_tiles > 0;
+    if (prep) {
         const int threads = 256;
         const int n_counters = pl.pair ? 2 * pl.sk_tiles : pl.sk_tiles;
         const int64_t n = std::max<int64_t>(pool ? M : 0, n_counters);
@@ -495,7 +577,7 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
             pool ? out : nullptr, pool ? M : 0, p.counters, n_counters);
         if (cudaGetLastError() != cudaSuccess) return FLE_ERR_CUDA;
     }
-    if (dispatch(pl, ta, tb, to, p, s) != cudaSuccess) return FLE_ERR_CUDA;
+    if (dispatch(pl, ta, tb, to, p, prep, s) != cudaSuccess) return FLE_ERR_CUDA;
     if (sync_check_enabled()) return fle_device_status(stream);
     return FLE_OK;
 }

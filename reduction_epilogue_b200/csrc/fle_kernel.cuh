@@ -50,7 +50,7 @@ enum : int { kPrec3xTF32 = 0, kPrecTF32 = 1 };
 // Wait-site identifiers recorded with a timeout.
 enum : unsigned {
     kWhereProdEmpty = 1, kWhereMmaFull = 2, kWhereMmaAccEmpty = 3, kWhereEpiAccFull = 4,
-    kWhereConvFull = 5, kWhereDrain = 6, kWhereProdDrain = 7, kWhereTest = 9
+    kWhereConvFull = 5, kWhereDrain = 6, kWhereProdDrain = 7, kWhereFixup = 8, kWhereTest = 9
 };
 
 struct KParams {
@@ -144,11 +144,17 @@ __host__ __device__ __forceinline__ int sk_slot_of(int c, int64_t tsk, int64_t s
     return (tsk == gb / num_kb) ? 0 : 1;
 }
 
-template <int BN, int PREC, bool SWAP>
+// KPS: k-blocks per ring stage.  A stage is [A of k-block 0..KPS-1 | B of
+// k-block 0..KPS-1] (then the same again for the 3xTF32 low parts).  Two
+// k-blocks per stage halve the producer/MMA handoffs per byte: each stage
+// costs a fixed barrier round trip, which otherwise caps the bytes a CTA
+// moves per microsecond.
+template <int BN, int PREC, bool SWAP, int KPS = 1>
 struct Cfg {
-    static constexpr int kABytes = kBM * kBK * 4;
-    static constexpr int kBBytes = BN * kBK * 4;
-    static constexpr int kLoadBytes = kABytes + kBBytes;            // TMA bytes per stage
+    static constexpr int kABytes = kBM * kBK * 4;                    // A rows of one k-block
+    static constexpr int kBBytes = BN * kBK * 4;                     // B rows of one k-block
+    static constexpr int kKbBytes = kABytes + kBBytes;
+    static constexpr int kLoadBytes = KPS * kKbBytes;                // TMA bytes per full stage
     static constexpr int kStageBytes = kLoadBytes * (PREC == kPrec3xTF32 ? 2 : 1);
     // direct layout: one 32 x 32 fp32 staging tile per epilogue warp for TMA stores
     static constexpr int kEpiStageBytes = SWAP ? 0 : kEpiWarps * kEpiTileBytes;
@@ -161,6 +167,7 @@ struct Cfg {
     static constexpr int kSmemBytes =
         1024 /*align slack*/ + kStages * kStageBytes + kEpiStageBytes + kNumBars * 8 + 32;
     static_assert(kStages >= 2, "need at least two stages");
+    static_assert(KPS == 1 || KPS == 2, "one or two k-blocks per stage");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128 is a multiple of 16 in [16,256]");
     static_assert(kABytes % 1024 == 0 && kBBytes % 1024 == 0, "tiles must keep 1024-byte alignment");
     static_assert(kSmemBytes <= 232448, "exceeds 227 KB of shared memory per block");
@@ -341,6 +348,9 @@ __device__ __forceinline__ void epi_chunk(const KParams& p, const Unit& u, int r
             default: epi_store_swapped<kEpiNone>(p, n, m0, v); break;
         }
     }
+    // Stores above may branch per lane (TMA issue, bounds); the warp must be
+    // converged again for the next tcgen05.ld (.sync.aligned).
+    __syncwarp();
 }
 
 template <bool SWAP>
@@ -348,6 +358,32 @@ __device__ __forceinline__ void epi_finish(const KParams& p, const Unit& u, int 
     if constexpr (!SWAP) {
         const int64_t m = static_cast<int64_t>(u.ta) * kBM + r;
         if (p.kind == kEpiPoolMax && m < p.M && best > -INFINITY) atomic_max_f32(p.out + m, best);
+    }
+    __syncwarp();
+}
+
+// Waits until *counter >= target (other CTAs raise it with atomicAdd after
+// a __threadfence), reading it with acquire semantics.  Bounded like the
+// mbarrier waits: gives up on *abort or after timeout_ns (recording a
+// timeout at `where` and raising *abort).
+__device__ __forceinline__ bool wait_count_bounded(const unsigned* counter, unsigned target, volatile int* abort,
+                                                   uint64_t timeout_ns, unsigned where) {
+    uint64_t t0 = 0;
+    uint32_t spins = 0;
+    while (true) {
+        unsigned v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+        if (v >= target) return true;
+        if (*abort) return false;
+        if (t0 == 0) t0 = global_timer_ns();
+        if ((++spins & 15u) == 0u) {
+            if (global_timer_ns() - t0 > timeout_ns) {
+                record_error(8u, where);
+                *abort = 1;
+                return false;
+            }
+            __nanosleep(100);
+        }
     }
 }
 
@@ -359,15 +395,17 @@ __device__ __forceinline__ void epilogue_bar_sync() {
 // ----------------------------------------------------------------------------
 // The kernel
 // ----------------------------------------------------------------------------
-template <int BN, int PREC, bool SWAP>
+template <int BN, int PREC, bool SWAP, int KPS>
 __global__ void __launch_bounds__(kThreads, 1)
 fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmOut, const KParams p) {
-    using C = Cfg<BN, PREC, SWAP>;
+    using C = Cfg<BN, PREC, SWAP, KPS>;
     constexpr int S = C::kStages;
     constexpr uint32_t kIdesc = idesc_tf32(kBM, BN);
-    // k-blocks per TMEM accumulation chain (see the epilogue role)
+    // k-blocks per TMEM accumulation chain (see the epilogue role); a
+    // multiple of KPS, so that chains and stages start on the same k-block
     constexpr int kChunkKb = (PREC == kPrec3xTF32) ? 4 : (1 << 30);
+    static_assert(kChunkKb % KPS == 0, "accumulation chains hold whole stages");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -384,9 +422,9 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     auto bar_accf = [&](int b) { return smem_u32(bars + 3 * S + b); };
     auto bar_acce = [&](int b) { return smem_u32(bars + 3 * S + 2 + b); };
     const uint32_t bar_drain = smem_u32(bars + 3 * S + 4);
-    // stage s: [A hi | B hi | A lo | B lo]
+    // stage s: [A hi | B hi | A lo | B lo], each part KPS k-blocks
     auto sA = [&](int s) { return sbase + s * C::kStageBytes; };
-    auto sB = [&](int s) { return sbase + s * C::kStageBytes + C::kABytes; };
+    auto sB = [&](int s) { return sbase + s * C::kStageBytes + KPS * C::kABytes; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -411,6 +449,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
         tmem_relinquish();
     }
+    __syncwarp();  // warp 0 branched on thread 0 above
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
@@ -427,15 +466,18 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             sc.init(p, blockIdx.x, gridDim.x);
             Unit u;
             while (ok && sc.next(p, u)) {
-                for (int kb = u.kb0; kb < u.kb1; ++kb) {
+                for (int kb = u.kb0; kb < u.kb1; kb += KPS) {
+                    const int n = (u.kb1 - kb < KPS) ? u.kb1 - kb : KPS;  // k-blocks in this stage
                     if (!mbar_wait_bounded(bar_empty(stage), phase ^ 1u, abort_flag, p.timeout_ns,
                                            kWhereProdEmpty)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(bar_full(stage), C::kLoadBytes);
-                    tma_load_2d(sA(stage), &tmA, bar_full(stage), kb * kBK, u.ta * kBM);
-                    tma_load_2d(sB(stage), &tmB, bar_full(stage), kb * kBK, u.tb * BN);
+                    mbar_arrive_expect_tx(bar_full(stage), n * C::kKbBytes);
+                    for (int j = 0; j < n; ++j) {
+                        tma_load_2d(sA(stage) + j * C::kABytes, &tmA, bar_full(stage), (kb + j) * kBK, u.ta * kBM);
+                        tma_load_2d(sB(stage) + j * C::kBBytes, &tmB, bar_full(stage), (kb + j) * kBK, u.tb * BN);
+                    }
                     ++fills;
                     if (++stage == S) { stage = 0; phase ^= 1u; }
                 }
@@ -470,28 +512,31 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 }
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
-                for (int kb = kc; kb < kce; ++kb) {
+                for (int kb = kc; kb < kce; kb += KPS) {
+                    const int n = (kce - kb < KPS) ? kce - kb : KPS;  // k-blocks in this stage
                     const uint32_t wbar = (PREC == kPrec3xTF32) ? bar_conv(stage) : bar_full(stage);
                     if (!mbar_wait_bounded(wbar, phase, abort_flag, p.timeout_ns, kWhereMmaFull)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint64_t a_hi = smem_desc_sw128(sA(stage));
-                    const uint64_t b_hi = smem_desc_sw128(sB(stage));
+                    for (int j = 0; j < n; ++j) {
+                        const uint64_t a_hi = smem_desc_sw128(sA(stage) + j * C::kABytes);
+                        const uint64_t b_hi = smem_desc_sw128(sB(stage) + j * C::kBBytes);
 #pragma unroll
-                    for (int k = 0; k < kBK / kUmmaK; ++k) {
-                        // advance 8 fp32 = 32 bytes along K inside the swizzle atom
-                        const uint64_t koff = static_cast<uint64_t>(k * 2);
-                        const uint32_t acc = (kb > kc || k > 0) ? 1u : 0u;
-                        if constexpr (PREC == kPrec3xTF32) {
-                            const uint64_t a_lo = smem_desc_sw128(sA(stage) + C::kLoadBytes);
-                            const uint64_t b_lo = smem_desc_sw128(sB(stage) + C::kLoadBytes);
-                            mma_tf32(d_tmem, a_lo + koff, b_hi + koff, kIdesc, acc);
-                            mma_tf32(d_tmem, a_hi + koff, b_lo + koff, kIdesc, 1u);
-                            mma_tf32(d_tmem, a_hi + koff, b_hi + koff, kIdesc, 1u);
-                        } else {
-                            mma_tf32(d_tmem, a_hi + koff, b_hi + koff, kIdesc, acc);
+                        for (int k = 0; k < kBK / kUmmaK; ++k) {
+                            // advance 8 fp32 = 32 bytes along K inside the swizzle atom
+                            const uint64_t koff = static_cast<uint64_t>(k * 2);
+                            const uint32_t acc = (kb > kc || j > 0 || k > 0) ? 1u : 0u;
+                            if constexpr (PREC == kPrec3xTF32) {
+                                const uint64_t a_lo = smem_desc_sw128(sA(stage) + C::kLoadBytes + j * C::kABytes);
+                                const uint64_t b_lo = smem_desc_sw128(sB(stage) + C::kLoadBytes + j * C::kBBytes);
+                                mma_tf32(d_tmem, a_lo + koff, b_hi + koff, kIdesc, acc);
+                                mma_tf32(d_tmem, a_hi + koff, b_lo + koff, kIdesc, 1u);
+                                mma_tf32(d_tmem, a_hi + koff, b_hi + koff, kIdesc, 1u);
+                            } else {
+                                mma_tf32(d_tmem, a_hi + koff, b_hi + koff, kIdesc, acc);
+                            }
                         }
                     }
                     mma_commit(bar_empty(stage));
@@ -520,7 +565,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             sc.init(p, blockIdx.x, gridDim.x);
             Unit u;
             while (ok && sc.next(p, u)) {
-                for (int kb = u.kb0; kb < u.kb1; ++kb) {
+                for (int kb = u.kb0; kb < u.kb1; kb += KPS) {
                     int got = 0;
                     if (lane == 0)
                         got = mbar_wait_bounded(bar_full(stage), phase, abort_flag, p.timeout_ns, kWhereConvFull);
@@ -552,6 +597,9 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         }
     } else {
         // ------------------------------------------------------------ epilogue
+        // The stream-K counters and (kind (c)) out are set by the prep
+        // kernel just before this one, which may still be running.
+        griddep_wait();
         // Eight warps.  Warp w reads TMEM lane quadrant w % 4 (tile rows
         // 32*(w%4) .. +31; a warp may only touch its own quadrant) and one
         // half of the tile's 32-column chunks, so each SM sub-partition runs
@@ -599,6 +647,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 tc_fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_acce(buf));
+                __syncwarp();
                 buf ^= 1;
                 if (buf == 0) acc_phase ^= 1u;
             };
@@ -658,11 +707,11 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 #undef FLE_EPI_BODY
                 epi_finish<SWAP>(p, u, r, best);
                 if constexpr (!kRegAcc) release_acc();
-            } else {
-                // Park this CTA's fp32 partial tile in its workspace slot,
-                // column-major inside the tile (element (row, col) at
-                // col * 128 + row) so that a warp's lanes write 32 consecutive
-                // floats.
+            } else if (u.kb0 != 0) {
+                // Not the tile's finisher: park this CTA's fp32 partial tile in
+                // its workspace slot, column-major inside the tile (element
+                // (row, col) at col * 128 + row) so that a warp's lanes write
+                // 32 consecutive floats, then count it on the tile's counter.
                 float* slot = p.ws + static_cast<size_t>(2 * blockIdx.x + u.slot) * kBM * BN;
 #define FLE_PARK_BODY(lc)                                                                 \
     {                                                                                     \
@@ -681,69 +730,89 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 }
 #undef FLE_PARK_BODY
                 if constexpr (!kRegAcc) release_acc();
-                const int64_t tsk = u.sk_tile;
-                const int first = sk_cta_of(tsk * p.num_kb, p.sk_iters, p.sk_grid);
-                const int last = sk_cta_of((tsk + 1) * p.num_kb - 1, p.sk_iters, p.sk_grid);
                 __threadfence();
                 epilogue_bar_sync();
-                if (threadIdx.x == 128) {
-                    const unsigned prev = atomicAdd(p.counters + tsk, 1u);
-                    *last_flag = (prev == static_cast<unsigned>(last - first)) ? 1 : 0;
-                }
+                if (threadIdx.x == 128) atomicAdd(p.counters + u.sk_tile, 1u);
+                __syncwarp();
+            } else {
+                // The tile's finisher: this unit holds k-block 0, the last unit
+                // of this CTA (its range ends inside the tile), while the other
+                // contributors ran the tile's later k-blocks as their first
+                // units.  Wait until all of them have parked their partials,
+                // then add them to this CTA's own accumulator in CTA order
+                // (= k order: a fixed order, so results are reproducible) and
+                // run the epilogue on the sum.
+                const int64_t tsk = u.sk_tile;
+                const int first = static_cast<int>(blockIdx.x);
+                const int last = sk_cta_of((tsk + 1) * p.num_kb - 1, p.sk_iters, p.sk_grid);
+                if (threadIdx.x == 128)
+                    *last_flag = wait_count_bounded(p.counters + tsk, static_cast<unsigned>(last - first),
+                                                    abort_flag, p.timeout_ns, kWhereFixup)
+                                     ? 1 : 0;
+                __syncwarp();  // named barriers are .aligned: whole warps arrive
                 epilogue_bar_sync();
-                if (*last_flag) {
-                    // Last to arrive: sum every contributor's partial in CTA
-                    // order (= k order), then run the epilogue on the sum.
-                    __threadfence();
-                    float best = -INFINITY;
+                const bool have = *last_flag != 0;
+                __threadfence();
+                float best = -INFINITY;
+                auto src_of = [&](int cc, int c) {
+                    const int sl = sk_slot_of(cc, tsk, p.sk_iters, p.sk_grid, p.num_kb);
+                    return p.ws + static_cast<size_t>(2 * cc + sl) * kBM * BN + static_cast<size_t>(c * 32) * kBM + r;
+                };
+                // own accumulator, then contributors first+1 .. last; loads of
+                // up to three contributors are in flight together
+#define FLE_FIX_BODY(lc)                                                                      \
+    {                                                                                         \
+        const int c = c_lo + (lc);                                                            \
+        float v[32];                                                                          \
+        FLE_LOAD_ACC(lc, v);                                                                  \
+        int cc = first + 1;                                                                   \
+        for (; cc + 2 <= last; cc += 3) {                                                     \
+            const float* s0 = src_of(cc, c);                                                  \
+            const float* s1 = src_of(cc + 1, c);                                              \
+            const float* s2 = src_of(cc + 2, c);                                              \
+            float t0[32], t1[32], t2[32];                                                     \
+            _Pragma("unroll") for (int j = 0; j < 32; ++j) {                                  \
+                t0[j] = __ldcg(s0 + j * kBM);                                                 \
+                t1[j] = __ldcg(s1 + j * kBM);                                                 \
+                t2[j] = __ldcg(s2 + j * kBM);                                                 \
+            }                                                                                 \
+            _Pragma("unroll") for (int j = 0; j < 32; ++j) v[j] = ((v[j] + t0[j]) + t1[j]) + t2[j]; \
+        }                                                                                     \
+        for (; cc <= last; ++cc) {                                                            \
+            const float* s0 = src_of(cc, c);                                                  \
+            float t0[32];                                                                     \
+            _Pragma("unroll") for (int j = 0; j < 32; ++j) t0[j] = __ldcg(s0 + j * kBM);      \
+            _Pragma("unroll") for (int j = 0; j < 32; ++j) v[j] += t0[j];                     \
+        }                                                                                     \
+        epi_chunk<SWAP, BN>(p, u, r, c, v, best, eo);                                         \
+    }
+                if (have) {
+                    if constexpr (kRegAcc) {
+#pragma unroll
+                        for (int lc = 0; lc < kHalf; ++lc)
+                            if (lc < mine) FLE_FIX_BODY(lc)
+                    } else {
 #pragma unroll 1
-                    for (int lc = 0; lc < mine; ++lc) {
-                        const int c = c_lo + lc;
-                        float v[32];
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = 0.0f;
-                        // Contributors in CTA order; loads of up to three
-                        // contributors are in flight together.
-                        auto src_of = [&](int cc) {
-                            const int sl = sk_slot_of(cc, tsk, p.sk_iters, p.sk_grid, p.num_kb);
-                            return p.ws + static_cast<size_t>(2 * cc + sl) * kBM * BN +
-                                   static_cast<size_t>(c * 32) * kBM + r;
-                        };
-                        int cc = first;
-                        for (; cc + 2 <= last; cc += 3) {
-                            const float* s0 = src_of(cc);
-                            const float* s1 = src_of(cc + 1);
-                            const float* s2 = src_of(cc + 2);
-                            float t0[32], t1[32], t2[32];
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) {
-                                t0[j] = __ldcg(s0 + j * kBM);
-                                t1[j] = __ldcg(s1 + j * kBM);
-                                t2[j] = __ldcg(s2 + j * kBM);
-                            }
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) v[j] = ((v[j] + t0[j]) + t1[j]) + t2[j];
-                        }
-                        for (; cc <= last; ++cc) {
-                            const float* s0 = src_of(cc);
-                            float t0[32];
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) t0[j] = __ldcg(s0 + j * kBM);
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) v[j] += t0[j];
-                        }
-                        epi_chunk<SWAP, BN>(p, u, r, c, v, best, eo);
+                        for (int lc = 0; lc < mine; ++lc) FLE_FIX_BODY(lc)
                     }
                     epi_finish<SWAP>(p, u, r, best);
-                    if (threadIdx.x == 128) p.counters[tsk] = 0u;
                 }
+#undef FLE_FIX_BODY
+                if constexpr (!kRegAcc) release_acc();
+                if (threadIdx.x == 128 && have) p.counters[tsk] = 0u;
+                __syncwarp();
+                if (!have) ok = false;
             }
 #undef FLE_LOAD_ACC
         }
     }
 
+    // Roles branch on the lane (one issuing thread per warp); reconverge every
+    // warp before the CTA barrier, which whole warps must reach together.
+    __syncwarp();
     // Epilogue TMA stores read the staging tiles until they complete.
     if (warp >= 4 && lane == 0) bulk_wait_all();
+    __syncwarp();
     tc_fence_before_sync();
     __syncthreads();
     if (warp == 1) {
@@ -782,6 +851,9 @@ __global__ void fle_bias_only_kernel(const KParams p) {
 // kind (the row maximum is combined with atomics) and zeroed stream-K
 // arrival counters.
 __global__ void fle_prep_kernel(float* fill, int64_t n_fill, unsigned* counters, int n_counters) {
+    // The GEMM that follows touches these words only after griddep_wait(),
+    // so it may be launched (and load its first tiles) right away.
+    griddep_launch_dependents();
     const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (fill != nullptr && i < n_fill) fill[i] = -INFINITY;
     if (counters != nullptr && i < n_counters) counters[i] = 0u;

@@ -27,36 +27,47 @@
 
 namespace fle {
 
-constexpr int kPairBN = 256;  // pair tile N (B rows)
+constexpr int kPairBN = 256;  // pair tile N (B rows), direct operand order
 constexpr int kPairBM = 256;  // pair tile M (A rows)
 
-template <int PREC>
+// KPS: k-blocks per ring stage, as in Cfg: [A k-blocks | B k-blocks].
+// BN: B rows of the pair tile (each CTA loads BN / 2 of them).  SWAP: A = W
+// and B = x, for the skinny shapes (BN = 32, 64, 128 covers M).
+template <int PREC, int KPS = 1, int BN = kPairBN, bool SWAP = false>
 struct PairCfg {
     static constexpr int kBKW = kBK;  // k-block width: 32 fp32, one 128-byte swizzle row
-    static constexpr int kABytes = kBM * kBKW * 4;            // this CTA's 128 A rows
-    static constexpr int kBBytes = (kPairBN / 2) * kBKW * 4;  // this CTA's 128 B rows
-    static constexpr int kLoadBytes = kABytes + kBBytes;      // TMA bytes per stage and CTA
+    static constexpr int kABytes = kBM * kBKW * 4;            // this CTA's 128 A rows, one k-block
+    static constexpr int kBBytes = (BN / 2) * kBKW * 4;       // this CTA's BN / 2 B rows, one k-block
+    static constexpr int kKbBytes = kABytes + kBBytes;
+    static constexpr int kLoadBytes = KPS * kKbBytes;         // TMA bytes per full stage and CTA
     static constexpr int kStageBytes = kLoadBytes * (PREC == kPrec3xTF32 ? 2 : 1);
-    static constexpr int kEpiStageBytes = kEpiWarps * kEpiTileBytes;  // TMA-store staging
-    static constexpr int kStages = (kSmemStageBudget - kEpiStageBytes) / kStageBytes;
-    static constexpr int kTmemCols = 512;                     // 2 accumulator buffers x 256 columns
+    // direct layout: TMA-store staging, one 32 x 32 tile per epilogue warp
+    static constexpr int kEpiStageBytes = SWAP ? 0 : kEpiWarps * kEpiTileBytes;
+    static constexpr int kStagesRaw = (kSmemStageBudget - kEpiStageBytes) / kStageBytes;
+    static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
+    static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
+                                    : (2 * BN <= 256) ? 256 : 512;  // 2 accumulator buffers x BN columns
     // full, split, empty per stage; accf, acce per buffer; drain; exit
     static constexpr int kNumBars = 3 * kStages + 4 + 2;
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kEpiStageBytes + kNumBars * 8 + 32;
     static_assert(kStages >= 2, "need at least two stages");
+    static_assert(KPS == 1 || KPS == 2, "one or two k-blocks per stage");
+    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "pair tile N: 32..256, whole 32-column chunks");
+    static_assert(kBBytes % 1024 == 0, "B halves keep 1024-byte alignment");
     static_assert(kSmemBytes <= 232448, "exceeds 227 KB of shared memory per block");
 };
 
-template <int PREC>
+template <int PREC, int KPS, int BN, bool SWAP>
 __global__ void __launch_bounds__(kThreads, 1)
 fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmOut, const KParams p) {
-    using C = PairCfg<PREC>;
+    using C = PairCfg<PREC, KPS, BN, SWAP>;
     constexpr bool k3x = (PREC == kPrec3xTF32);
     constexpr int S = C::kStages;
-    constexpr uint32_t kIdesc = idesc_tf32(kPairBM, kPairBN);
+    constexpr uint32_t kIdesc = idesc_tf32(kPairBM, BN);
     constexpr int kBKW = C::kBKW;
     constexpr int kChunkKb = k3x ? 128 / kBKW : (1 << 30);  // k-blocks per TMEM accumulation chain
+    static_assert(kChunkKb % KPS == 0, "accumulation chains hold whole stages");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -76,7 +87,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     const uint32_t bar_exit = smem_u32(bars + 3 * S + 5);
     // stage s: [A | B | A lo | B lo]; the lo half exists for 3xTF32 only
     auto sA = [&](int s) { return sbase + s * C::kStageBytes; };
-    auto sB = [&](int s) { return sbase + s * C::kStageBytes + C::kABytes; };
+    auto sB = [&](int s) { return sbase + s * C::kStageBytes + KPS * C::kABytes; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -105,6 +116,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         tmem_alloc_pair(smem_u32(tmem_slot), C::kTmemCols);
         tmem_relinquish_pair();
     }
+    __syncwarp();  // warp 0 branched on thread 0 above
     tc_fence_before_sync();
     cluster_sync_all();  // both CTAs' barriers exist before either signals the other
     tc_fence_after_sync();
@@ -121,25 +133,30 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             sc.init(p, pair, num_pairs);
             Unit u;
             while (ok && sc.next(p, u)) {
-                for (int kb = u.kb0; kb < u.kb1; ++kb) {
+                const int32_t ra = u.ta * kPairBM + static_cast<int32_t>(rank) * kBM;
+                const int32_t rb = u.tb * BN + static_cast<int32_t>(rank) * (BN / 2);
+                for (int kb = u.kb0; kb < u.kb1; kb += KPS) {
+                    const int n = (u.kb1 - kb < KPS) ? u.kb1 - kb : KPS;  // k-blocks in this stage
                     if (!mbar_wait_bounded(bar_empty(stage), phase ^ 1u, abort_flag, p.timeout_ns,
                                            kWhereProdEmpty)) {
                         ok = false;
                         break;
                     }
-                    const int32_t ra = u.ta * kPairBM + static_cast<int32_t>(rank) * kBM;
-                    const int32_t rb = u.tb * kPairBN + static_cast<int32_t>(rank) * (kPairBN / 2);
                     if constexpr (k3x) {
                         // own barrier: this CTA's split warps wait for these bytes
-                        mbar_arrive_expect_tx(bar_full(stage), C::kLoadBytes);
-                        tma_load_2d(sA(stage), &tmA, bar_full(stage), kb * kBKW, ra);
-                        tma_load_2d(sB(stage), &tmB, bar_full(stage), kb * kBKW, rb);
+                        mbar_arrive_expect_tx(bar_full(stage), n * C::kKbBytes);
+                        for (int j = 0; j < n; ++j) {
+                            tma_load_2d(sA(stage) + j * C::kABytes, &tmA, bar_full(stage), (kb + j) * kBKW, ra);
+                            tma_load_2d(sB(stage) + j * C::kBBytes, &tmB, bar_full(stage), (kb + j) * kBKW, rb);
+                        }
                     } else {
                         // the leader expects both CTAs' bytes on its own full barrier
-                        if (rank == 0) mbar_arrive_expect_tx(bar_full(stage), 2 * C::kLoadBytes);
+                        if (rank == 0) mbar_arrive_expect_tx(bar_full(stage), 2 * n * C::kKbBytes);
                         const uint32_t leader_full = mapa_shared(bar_full(stage), 0);
-                        tma_load_2d_pair(sA(stage), &tmA, leader_full, kb * kBKW, ra);
-                        tma_load_2d_pair(sB(stage), &tmB, leader_full, kb * kBKW, rb);
+                        for (int j = 0; j < n; ++j) {
+                            tma_load_2d_pair(sA(stage) + j * C::kABytes, &tmA, leader_full, (kb + j) * kBKW, ra);
+                            tma_load_2d_pair(sB(stage) + j * C::kBBytes, &tmB, leader_full, (kb + j) * kBKW, rb);
+                        }
                     }
                     ++fills;
                     if (++stage == S) { stage = 0; phase ^= 1u; }
@@ -174,8 +191,9 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kPairBN);
-                    for (int kb = kc; kb < kce; ++kb) {
+                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+                    for (int kb = kc; kb < kce; kb += KPS) {
+                        const int n = (kce - kb < KPS) ? kce - kb : KPS;  // k-blocks in this stage
                         const uint32_t wbar = k3x ? bar_split(stage) : bar_full(stage);
                         if (!mbar_wait_bounded(wbar, phase, abort_flag, p.timeout_ns, kWhereMmaFull)) {
                             ok = false;
@@ -183,21 +201,23 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                         }
                         tc_fence_after_sync();
                         auto desc = [](uint32_t a) { return smem_desc_sw128(a); };
-                        const uint64_t a_hi = desc(sA(stage));
-                        const uint64_t b_hi = desc(sB(stage));
+                        for (int j = 0; j < n; ++j) {
+                            const uint64_t a_hi = desc(sA(stage) + j * C::kABytes);
+                            const uint64_t b_hi = desc(sB(stage) + j * C::kBBytes);
 #pragma unroll
-                        for (int k = 0; k < kBKW / kUmmaK; ++k) {
-                            // advance 8 fp32 = 32 bytes along K inside the swizzle atom
-                            const uint64_t koff = static_cast<uint64_t>(k * 2);
-                            const uint32_t acc = (kb > kc || k > 0) ? 1u : 0u;
-                            if constexpr (k3x) {
-                                const uint64_t a_lo = desc(sA(stage) + C::kLoadBytes);
-                                const uint64_t b_lo = desc(sB(stage) + C::kLoadBytes);
-                                mma_tf32_pair(d_tmem, a_lo + koff, b_hi + koff, kIdesc, acc);
-                                mma_tf32_pair(d_tmem, a_hi + koff, b_lo + koff, kIdesc, 1u);
-                                mma_tf32_pair(d_tmem, a_hi + koff, b_hi + koff, kIdesc, 1u);
-                            } else {
-                                mma_tf32_pair(d_tmem, a_hi + koff, b_hi + koff, kIdesc, acc);
+                            for (int k = 0; k < kBKW / kUmmaK; ++k) {
+                                // advance 8 fp32 = 32 bytes along K inside the swizzle atom
+                                const uint64_t koff = static_cast<uint64_t>(k * 2);
+                                const uint32_t acc = (kb > kc || j > 0 || k > 0) ? 1u : 0u;
+                                if constexpr (k3x) {
+                                    const uint64_t a_lo = desc(sA(stage) + C::kLoadBytes + j * C::kABytes);
+                                    const uint64_t b_lo = desc(sB(stage) + C::kLoadBytes + j * C::kBBytes);
+                                    mma_tf32_pair(d_tmem, a_lo + koff, b_hi + koff, kIdesc, acc);
+                                    mma_tf32_pair(d_tmem, a_hi + koff, b_lo + koff, kIdesc, 1u);
+                                    mma_tf32_pair(d_tmem, a_hi + koff, b_hi + koff, kIdesc, 1u);
+                                } else {
+                                    mma_tf32_pair(d_tmem, a_hi + koff, b_hi + koff, kIdesc, acc);
+                                }
                             }
                         }
                         mma_commit_pair_multicast(bar_empty(stage), 0x3);
@@ -225,7 +245,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             sc.init(p, pair, num_pairs);
             Unit u;
             while (ok && sc.next(p, u)) {
-                for (int kb = u.kb0; kb < u.kb1; ++kb) {
+                for (int kb = u.kb0; kb < u.kb1; kb += KPS) {
                     int got = 0;
                     if (lane == 0)
                         got = mbar_wait_bounded(bar_full(stage), phase, abort_flag, p.timeout_ns, kWhereConvFull);
@@ -251,15 +271,19 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         }
     } else {
         // ------------------------------------------------------------ epilogue (both CTAs)
+        // The stream-K counters and (kind (c)) out are set by the prep
+        // kernel just before this one, which may still be running.
+        griddep_wait();
         // Eight warps: lane quadrant warp % 4, half of the columns each.
         const int q = warp & 3;
         const int half = (warp - 4) >> 2;
         const int r = q * 32 + lane;
-        constexpr int kHalf = kPairBN / 32 / 2;  // chunks per half
+        constexpr int kChunks = BN / 32;
+        constexpr int kHalf = (kChunks + 1) / 2;  // chunks per half
         const int c_lo = half * kHalf;
         EpiOut eo;
-        eo.tmap = p.tma_out ? &tmOut : nullptr;
-        eo.stage = reinterpret_cast<float*>(epi_stage + (warp - 4) * kEpiTileBytes);
+        eo.tmap = (!SWAP && p.tma_out) ? &tmOut : nullptr;
+        eo.stage = reinterpret_cast<float*>(epi_stage + (SWAP ? 0 : (warp - 4) * kEpiTileBytes));
         eo.stage_u32 = smem_u32(eo.stage);
         int buf = 0;
         uint32_t acc_phase = 0;
@@ -269,8 +293,8 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         Unit u;
         bool ok = true;
         while (ok && sc.next(p, u)) {
-            const int64_t cols_left = p.N - static_cast<int64_t>(u.tb) * kPairBN;
-            const int nchunks = static_cast<int>(cols_left >= kPairBN ? kPairBN / 32 : (cols_left + 31) / 32);
+            const int64_t cols_left = (SWAP ? p.M : p.N) - static_cast<int64_t>(u.tb) * BN;
+            const int nchunks = static_cast<int>(cols_left >= BN ? kChunks : (cols_left + 31) / 32);
             const int mine = nchunks - c_lo < 0 ? 0 : (nchunks - c_lo > kHalf ? kHalf : nchunks - c_lo);
             // This CTA's 128 rows of the pair tile, as a 128-row tile index.
             Unit uh = u;
@@ -288,11 +312,12 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 tc_fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(mapa_shared(bar_acce(buf), 0));
+                __syncwarp();
                 buf ^= 1;
                 if (buf == 0) acc_phase ^= 1u;
             };
             auto t_row = [&]() {
-                return tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * kPairBN);
+                return tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * BN);
             };
 
             uint32_t t_acc = 0;
@@ -330,7 +355,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                             float v[32];
 #pragma unroll
                             for (int j = 0; j < 32; ++j) v[j] = accr[lc * 32 + j];
-                            epi_chunk<false, kPairBN>(p, uh, r, c_lo + lc, v, best, eo);
+                            epi_chunk<SWAP, BN>(p, uh, r, c_lo + lc, v, best, eo);
                         }
                     }
                 } else {
@@ -338,14 +363,15 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     for (int lc = 0; lc < mine; ++lc) {
                         float v[32];
                         tmem_ld32_wait(t_acc + (c_lo + lc) * 32, v);
-                        epi_chunk<false, kPairBN>(p, uh, r, c_lo + lc, v, best, eo);
+                        epi_chunk<SWAP, BN>(p, uh, r, c_lo + lc, v, best, eo);
                     }
                 }
-                epi_finish<false>(p, uh, r, best);
+                epi_finish<SWAP>(p, uh, r, best);
                 if constexpr (!k3x) release_acc();
-            } else {
-                // column-major partial tile: element (row, col) at col * 128 + row
-                float* slot = p.ws + static_cast<size_t>(2 * blockIdx.x + u.slot) * kBM * kPairBN;
+            } else if (u.kb0 != 0) {
+                // Not the tile's finisher: park this CTA's partial (column-major:
+                // element (row, col) at col * 128 + row) and count it.
+                float* slot = p.ws + static_cast<size_t>(2 * blockIdx.x + u.slot) * kBM * BN;
                 if constexpr (k3x) {
 #pragma unroll
                     for (int lc = 0; lc < kHalf; ++lc) {
@@ -366,67 +392,97 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     }
                     release_acc();
                 }
-                const int64_t tsk = u.sk_tile;
-                const int first = sk_cta_of(tsk * p.num_kb, p.sk_iters, p.sk_grid);
-                const int last = sk_cta_of((tsk + 1) * p.num_kb - 1, p.sk_iters, p.sk_grid);
-                unsigned* counter = p.counters + 2 * tsk + rank;
                 __threadfence();
                 epilogue_bar_sync();
-                if (threadIdx.x == 128) {
-                    const unsigned prev = atomicAdd(counter, 1u);
-                    *last_flag = (prev == static_cast<unsigned>(last - first)) ? 1 : 0;
-                }
+                if (threadIdx.x == 128) atomicAdd(p.counters + 2 * u.sk_tile + rank, 1u);
+                __syncwarp();
+            } else {
+                // The tile's finisher (this pair's last unit holds k-block 0):
+                // wait for the other pairs' partials of this CTA's 128 rows,
+                // add them to the own accumulator in pair order (= k order),
+                // then run the epilogue.
+                const int64_t tsk = u.sk_tile;
+                const int first = pair;
+                const int last = sk_cta_of((tsk + 1) * p.num_kb - 1, p.sk_iters, p.sk_grid);
+                unsigned* counter = p.counters + 2 * tsk + rank;
+                if (threadIdx.x == 128)
+                    *last_flag = wait_count_bounded(counter, static_cast<unsigned>(last - first), abort_flag,
+                                                    p.timeout_ns, kWhereFixup)
+                                     ? 1 : 0;
+                __syncwarp();  // named barriers are .aligned: whole warps arrive
                 epilogue_bar_sync();
-                if (*last_flag) {
-                    __threadfence();
-                    float best = -INFINITY;
-#pragma unroll 1
-                    for (int lc = 0; lc < mine; ++lc) {
-                        const int c = c_lo + lc;
-                        float v[32];
+                const bool have = *last_flag != 0;
+                __threadfence();
+                float best = -INFINITY;
+                auto src_of = [&](int cc, int c) {
+                    const int sl = sk_slot_of(cc, tsk, p.sk_iters, p.sk_grid, p.num_kb);
+                    return p.ws + static_cast<size_t>(2 * (2 * cc + rank) + sl) * kBM * BN +
+                           static_cast<size_t>(c * 32) * kBM + r;
+                };
+                // contributors first+1 .. last after the own accumulator; loads
+                // of up to three contributors are in flight together
+                auto add_partials = [&](int c, float (&v)[32]) {
+                    int cc = first + 1;
+                    for (; cc + 2 <= last; cc += 3) {
+                        const float* s0 = src_of(cc, c);
+                        const float* s1 = src_of(cc + 1, c);
+                        const float* s2 = src_of(cc + 2, c);
+                        float t0[32], t1[32], t2[32];
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = 0.0f;
-                        // Contributors in CTA order; loads of up to three
-                        // contributors are in flight together.
-                        auto src_of = [&](int cc) {
-                            const int sl = sk_slot_of(cc, tsk, p.sk_iters, p.sk_grid, p.num_kb);
-                            return p.ws + static_cast<size_t>(2 * (2 * cc + rank) + sl) * kBM * kPairBN +
-                                   static_cast<size_t>(c * 32) * kBM + r;
-                        };
-                        int cc = first;
-                        for (; cc + 2 <= last; cc += 3) {
-                            const float* s0 = src_of(cc);
-                            const float* s1 = src_of(cc + 1);
-                            const float* s2 = src_of(cc + 2);
-                            float t0[32], t1[32], t2[32];
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) {
-                                t0[j] = __ldcg(s0 + j * kBM);
-                                t1[j] = __ldcg(s1 + j * kBM);
-                                t2[j] = __ldcg(s2 + j * kBM);
-                            }
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) v[j] = ((v[j] + t0[j]) + t1[j]) + t2[j];
+                        for (int j = 0; j < 32; ++j) {
+                            t0[j] = __ldcg(s0 + j * kBM);
+                            t1[j] = __ldcg(s1 + j * kBM);
+                            t2[j] = __ldcg(s2 + j * kBM);
                         }
-                        for (; cc <= last; ++cc) {
-                            const float* s0 = src_of(cc);
-                            float t0[32];
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) t0[j] = __ldcg(s0 + j * kBM);
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) v[j] += t0[j];
-                        }
-                        epi_chunk<false, kPairBN>(p, uh, r, c, v, best, eo);
+                        for (int j = 0; j < 32; ++j) v[j] = ((v[j] + t0[j]) + t1[j]) + t2[j];
                     }
-                    epi_finish<false>(p, uh, r, best);
-                    if (threadIdx.x == 128) *counter = 0u;
+                    for (; cc <= last; ++cc) {
+                        const float* s0 = src_of(cc, c);
+                        float t0[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) t0[j] = __ldcg(s0 + j * kBM);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] += t0[j];
+                    }
+                };
+                if (have) {
+                    if constexpr (k3x) {
+#pragma unroll
+                        for (int lc = 0; lc < kHalf; ++lc) {
+                            if (lc < mine) {
+                                float v[32];
+#pragma unroll
+                                for (int j = 0; j < 32; ++j) v[j] = accr[lc * 32 + j];
+                                add_partials(c_lo + lc, v);
+                                epi_chunk<SWAP, BN>(p, uh, r, c_lo + lc, v, best, eo);
+                            }
+                        }
+                    } else {
+#pragma unroll 1
+                        for (int lc = 0; lc < mine; ++lc) {
+                            float v[32];
+                            tmem_ld32_wait(t_acc + (c_lo + lc) * 32, v);
+                            add_partials(c_lo + lc, v);
+                            epi_chunk<SWAP, BN>(p, uh, r, c_lo + lc, v, best, eo);
+                        }
+                    }
+                    epi_finish<SWAP>(p, uh, r, best);
                 }
+                if constexpr (!k3x) release_acc();
+                if (threadIdx.x == 128 && have) *counter = 0u;
+                __syncwarp();
+                if (!have) ok = false;
             }
         }
     }
 
+    // Roles branch on the lane (one issuing thread per warp); reconverge every
+    // warp before the CTA barriers, which whole warps must reach together.
+    __syncwarp();
     // Epilogue TMA stores read the staging tiles until they complete.
     if (warp >= 4 && lane == 0) bulk_wait_all();
+    __syncwarp();
     // Neither CTA may release TMEM or exit while the other can still signal
     // its barriers or (leader) write its TMEM: a bounded two-way handshake.
     tc_fence_before_sync();
@@ -436,6 +492,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         volatile int never = 0;
         mbar_wait_bounded(bar_exit, 0, &never, p.timeout_ns, kWhereDrain);
     }
+    __syncwarp();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after_sync();

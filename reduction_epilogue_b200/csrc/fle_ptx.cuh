@@ -23,6 +23,16 @@ __device__ __forceinline__ void record_error(unsigned code, unsigned where) {
     atomicAdd(&g_status[3], 1u);
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start before the previous kernel in the stream ends;
+// griddep_wait() blocks the calling thread until that kernel has completed
+// and its writes are visible, and griddep_launch_dependents() lets the next
+// kernel start early.  Both are no-ops for an ordinary launch.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -280,12 +280,15 @@ def test_long_k_accuracy_3xtf32(fle, precision):
 def test_epilogue_math_against_fp64_and_cuda(fle, which):
     # The epilogue evaluates erf by Abramowitz & Stegun 7.1.26 (|error| <=
     # 1.5e-7) and the sigmoid with a fast exponential and divide; bound both
-    # against fp64 and against CUDA's erff / expf on a dense grid.
+    # against fp64 and against CUDA's erff / expf on a dense grid and at
+    # saturating magnitudes.
     from scipy.special import erf as erf64
     lib = fle.load()
     lib.fle_test_epilogue_math.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32,
                                            ctypes.c_int32, ctypes.c_void_p]
-    xs = torch.linspace(-9.0, 9.0, 360001, device="cuda")
+    # a dense grid plus magnitudes where exp over- or underflows in fp32
+    extremes = torch.tensor([-1e4, -500.0, -100.0, -88.0, -50.0, 50.0, 88.0, 100.0, 500.0, 1e4])
+    xs = torch.cat([torch.linspace(-9.0, 9.0, 360001), extremes]).cuda()
     got = torch.empty_like(xs)
     cuda_ref = torch.empty_like(xs)
     assert lib.fle_test_epilogue_math(xs.data_ptr(), got.data_ptr(), xs.numel(), which, 0, None) == 0
@@ -306,3 +309,62 @@ def test_epilogue_math_against_fp64_and_cuda(fle, which):
     assert np.isfinite(g).all()
     assert np.abs(g - exact).max() <= bound.max() and (np.abs(g - exact) <= bound).all()
     assert (np.abs(g - c) <= 2 * bound).all()
+
+
+_STAGE_VARIANT_SCRIPT = r"""
+import sys, numpy as np, torch
+import oracle
+import reduction_epilogue_b200 as fle
+from reduction_epilogue_b200 import synth
+fle.load()
+bad = []
+for (M, K, N, problem) in [(16, 2080, 300, "scale_hardtanh_gelu"), (100, 1056, 520, "swish_scale"),
+                           (300, 1056, 600, "scale_hardtanh_gelu"), (520, 2080, 1100, "avgpool_gelu_scale_rowmax"),
+                           (33, 20000, 3000, "none")]:
+    x, W, b = synth.linear_inputs(M, K, N, seed=7, device="cuda")
+    out = fle.linear_epilogue(x, W, b, problem, "tf32")
+    torch.cuda.synchronize()
+    rows = synth.sample_rows(M, 24, seed=3)
+    ref = oracle.forward_rows(x.cpu().numpy(), W.cpu().numpy(), b.cpu().numpy(), rows=rows,
+                              **oracle.PROBLEMS[problem]).astype(np.float64)
+    got = out.cpu().numpy()[rows].astype(np.float64)
+    err = np.abs(got - ref) - (5e-3 + 5e-3 * np.abs(ref))
+    if fle.device_status() != 0 or not np.isfinite(got).all() or (err > 0).any():
+        bad.append((M, K, N, problem, float(err.max())))
+print("PLAN", fle.plan_string(300, 1056, 600, fle.desc_for("scale_hardtanh_gelu", "tf32")))
+print("BAD", bad)
+sys.exit(1 if bad else 0)
+"""
+
+
+@pytest.mark.parametrize("kps", ["1", "2"])
+def test_one_and_two_kblocks_per_stage(fle, kps):
+    # Ring stages hold one or two 32-wide k-blocks (the planner picks per
+    # plan; FLE_KPS forces one).  Both forms, in both kernels and with odd
+    # k-block counts per unit (K = 1056, 2080 and 20000 are 33, 65 and 625
+    # k-blocks), against the oracle, in a fresh process.
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, FLE_KPS=kps, PYTHONPATH=root)
+    r = subprocess.run([sys.executable, "-c", _STAGE_VARIANT_SCRIPT], cwd=root, env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert f"kps={kps}" in r.stdout
+
+
+@pytest.mark.parametrize("problem", ["scale_hardtanh_gelu", "swish_scale"])
+@pytest.mark.parametrize("M", [1, 45, 100, 128])
+def test_swapped_pair_tiles(fle, M, problem):
+    # Skinny M with at least one 256-row weight tile per CTA pair runs the
+    # swapped pair kernel (each CTA of a pair: 128 weight rows, half of the
+    # activation rows).  Ragged M (BN = 32, 64, 128), ragged N (75 tiles, the
+    # last one 93 rows short) and a ragged K tail.
+    M, K, N = M, 520, 75 * 256 - 93
+    d = fle.desc_for(problem, "tf32")
+    plan = fle.plan_string(M, K, N, d)
+    assert "pair=1 swap=1" in plan, plan
+    x, W, b = synth.linear_inputs(M, K, N, seed=11, device="cuda")
+    out = _run(fle, x, W, b, problem, "tf32")
+    _assert_close(out.cpu().numpy(), _oracle(x, W, b, problem), "tf32", f"{M}x{K}x{N} {plan}")

@@ -72,9 +72,9 @@ def test_schedule_covers_every_kblock_once(M, K, N, problem, precision, sms):
     tas = {e[3][0] for v in cover.values() for e in v}
     tbs = {e[3][1] for v in cover.values() for e in v}
     assert len(tas) * len(tbs) == len(tiles)
-    # the tiles span exactly the operand rows (A side holds M or N, in tiles
-    # of 128 rows, or 256 rows on CTA pairs)
-    a_rows = {math.ceil(M / 128), math.ceil(N / 128), math.ceil(M / 256)}
+    # the tiles span exactly the operand rows (A side holds M, or N in the
+    # swapped order, in tiles of 128 rows, or 256 rows on CTA pairs)
+    a_rows = {math.ceil(M / 128), math.ceil(N / 128), math.ceil(M / 256), math.ceil(N / 256)}
     assert len(tas) in a_rows
 
     for t, units in cover.items():
@@ -120,14 +120,30 @@ def test_headline_shape_splits_only_the_last_wave():
     assert grid3 == 74 and sum(int(r[4]) - int(r[3]) for rows in per3 for r in rows) == 256 * 256
 
 
-def test_weight_streamed_once_shapes_use_every_sm():
-    # M = 16 (swapped): 64 weight tiles, each read by one unit; all 148 SMs
-    # share the k-blocks evenly (to within one).
+def test_weight_streamed_once_shapes_split_each_tile():
+    # M = 16 (swapped): 64 weight tiles of 128 rows on 148 SMs; each tile is
+    # split into two k-aligned halves on 128 CTAs, every CTA streaming the
+    # same 128 k-blocks of one tile.
     desc = fle.desc_for("scale_hardtanh_gelu", "tf32")
     grid, per_cta = collect(16, 8192, 8192, desc, 148)
-    assert grid == 148
-    load = [sum(int(r[4]) - int(r[3]) for r in rows) for rows in per_cta]
-    assert max(load) - min(load) <= 1
+    assert grid == 128
+    units = [r for rows in per_cta for r in rows]
+    assert len(units) == 128
+    assert {(int(r[3]), int(r[4])) for r in units} == {(0, 128), (128, 256)}
+
+
+def test_skinny_weight_stream_runs_whole_tiles_on_pairs():
+    # 128 x 32768 x 32768 in TF32: 128 weight tiles of 256 rows on the 74
+    # CTA pairs, each tile streamed whole by one pair (measured faster than
+    # splitting the stream along K); 3xTF32 keeps one-CTA tiles of 128 rows.
+    desc = fle.desc_for("swish_scale", "tf32")
+    grid, per_cta = collect(128, 32768, 32768, desc, 148)
+    assert grid == 74
+    units = [r for rows in per_cta for r in rows]
+    assert len(units) == 128 and all(int(r[5]) == 0 for r in units)  # whole tiles, no partials
+    assert {(int(r[3]), int(r[4])) for r in units} == {(0, 1024)}
+    grid3, per3 = collect(128, 32768, 32768, fle.desc_for("swish_scale", "3xtf32"), 148)
+    assert grid3 == 148
 
 
 def test_workspace_matches_the_plan():
@@ -139,4 +155,4 @@ def test_workspace_matches_the_plan():
     g = ctypes.c_int(0)
     assert lib.fle_plan_units(128, 32768, 32768, ctypes.byref(desc), 148, 0, None, 0,
                               ctypes.byref(n), ctypes.byref(g)) == 0
-    assert g.value == 148
+    assert g.value == 74  # CTA pairs, whole tiles: no workspace
