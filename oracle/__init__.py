@@ -48,6 +48,8 @@ def _load():
     lib.orc_num_threads.restype = ctypes.c_int
     lib.orc_gelu.argtypes = [dbl]
     lib.orc_gelu.restype = dbl
+    lib.orc_gelu_tanh.argtypes = [dbl]
+    lib.orc_gelu_tanh.restype = dbl
     lib.orc_scale_hardtanh_gelu.argtypes = [dbl, dbl, dbl, dbl]
     lib.orc_scale_hardtanh_gelu.restype = dbl
     lib.orc_swish_scale.argtypes = [dbl, dbl]
@@ -59,7 +61,7 @@ def _load():
     lib.orc_linear_rows.argtypes = [vp, vp, vp, i64, i64, i64, vp, i64, vp]
     lib.orc_linear_rows.restype = None
     lib.orc_forward_rows.argtypes = [vp, vp, vp, i64, i64, i64, ctypes.c_int,
-                                     dbl, dbl, dbl, i64, i64, vp, i64, vp, vp]
+                                     dbl, dbl, dbl, i64, i64, ctypes.c_int, vp, i64, vp, vp]
     lib.orc_forward_rows.restype = ctypes.c_int
     _lib = lib
     return lib
@@ -80,6 +82,11 @@ def num_threads() -> int:
 
 def gelu(v: float) -> float:
     return float(_load().orc_gelu(float(v)))
+
+
+def gelu_tanh(v: float) -> float:
+    """GELU in its tanh form (page l2_p53's first fused kernel)."""
+    return float(_load().orc_gelu_tanh(float(v)))
 
 
 def scale_hardtanh_gelu(y: float, s: float = 0.5, lo: float = -2.0, hi: float = 2.0) -> float:
@@ -115,11 +122,11 @@ def linear_rows(x, W, b, rows=None) -> np.ndarray:
 
 def forward_rows(x, W, b, kind: int, scale: float = 1.0, clamp_lo: float = -2.0,
                  clamp_hi: float = 2.0, pool_k: int = 16, pool_stride: int | None = None,
-                 rows=None) -> np.ndarray:
+                 rows=None, gelu_tanh: bool = False) -> np.ndarray:
     """The whole path (linear + epilogue ``kind``) for the given rows, fp32 result.
 
     Returns [len(rows), N] for the elementwise kinds and [len(rows)] for the
-    pool / row-max kind.
+    pool / row-max kind.  gelu_tanh: GELU in its tanh form for (a) and (c).
     """
     x, W = _f32(x), _f32(W)
     b = None if b is None else _f32(b)
@@ -131,7 +138,7 @@ def forward_rows(x, W, b, kind: int, scale: float = 1.0, clamp_lo: float = -2.0,
     out = np.empty((R,) if kind == EPI_AVGPOOL_GELU_SCALE_ROWMAX else (R, N), dtype=np.float32)
     rc = _load().orc_forward_rows(_ptr(x), _ptr(W), _ptr(b), M, K, N, int(kind), float(scale),
                                   float(clamp_lo), float(clamp_hi), int(pool_k),
-                                  int(pool_k if pool_stride is None else pool_stride),
+                                  int(pool_k if pool_stride is None else pool_stride), int(bool(gelu_tanh)),
                                   _ptr(rows), R, _ptr(out), None)
     if rc != 0:
         raise ValueError("oracle rejected the arguments (rc=%d)" % rc)

@@ -32,6 +32,12 @@
  *              including its output-length check for N=8192, k=16).
  *   none    out = y  (the Linear alone; used to check the contraction itself).
  *
+ * Option (a), (c): GELU in its tanh form instead of the erf form,
+ *           GELU_tanh(v) = v/2 * (1 + tanh(sqrt(2/pi) * (v + 0.044715 v^3)))
+ *           -- the approximation page "Kimi-K2.6 l2_p53" writes into its first
+ *              fused elementwise kernel and then weighs against the exact form
+ *              (gelu_tanh = 1 below).
+ *
  * Build: gcc -O2 -fopenmp -fPIC -shared (no -ffast-math: the fp64
  * evaluation must not be reassociated).
  */
@@ -63,11 +69,24 @@ static double orc_phi(double v) { return 0.5 * (1.0 + erf(v / sqrt(2.0))); }
 /* Exact GELU: v * Phi(v) (PyTorch's default approximate='none'). */
 double orc_gelu(double v) { return v * orc_phi(v); }
 
+/* GELU in its tanh form: v/2 * (1 + tanh(sqrt(2/pi) * (v + 0.044715 v^3))). */
+double orc_gelu_tanh(double v) {
+    const double c = sqrt(2.0 / acos(-1.0));
+    return 0.5 * v * (1.0 + tanh(c * (v + 0.044715 * v * v * v)));
+}
+
+/* The GELU of the selected form (0: erf, 1: tanh). */
+static double orc_gelu_form(double v, int gelu_tanh) { return gelu_tanh ? orc_gelu_tanh(v) : orc_gelu(v); }
+
 /* Epilogue (a) on one linear output. */
-double orc_scale_hardtanh_gelu(double y, double s, double lo, double hi) {
+double orc_scale_hardtanh_gelu_form(double y, double s, double lo, double hi, int gelu_tanh) {
     double t = s * y;
     t = fmin(fmax(t, lo), hi);
-    return orc_gelu(t);
+    return orc_gelu_form(t, gelu_tanh);
+}
+
+double orc_scale_hardtanh_gelu(double y, double s, double lo, double hi) {
+    return orc_scale_hardtanh_gelu_form(y, s, lo, hi, 0);
 }
 
 /* Epilogue (b) on one linear output. */
@@ -83,18 +102,23 @@ int64_t orc_pool_windows(int64_t N, int64_t k, int64_t stride) {
 }
 
 /* Epilogue (c) on one full linear row y[0..N). */
-double orc_pool_gelu_scale_max(const double* yrow, int64_t N, int64_t k,
-                               int64_t stride, double s) {
+double orc_pool_gelu_scale_max_form(const double* yrow, int64_t N, int64_t k,
+                                    int64_t stride, double s, int gelu_tanh) {
     int64_t P = orc_pool_windows(N, k, stride);
     double best = -INFINITY;
     for (int64_t j = 0; j < P; ++j) {
         double acc = 0.0;
         for (int64_t t = 0; t < k; ++t) acc += yrow[j * stride + t];
         double p = acc / (double)k;
-        double g = s * orc_gelu(p);
+        double g = s * orc_gelu_form(p, gelu_tanh);
         if (g > best) best = g;
     }
     return best;
+}
+
+double orc_pool_gelu_scale_max(const double* yrow, int64_t N, int64_t k,
+                               int64_t stride, double s) {
+    return orc_pool_gelu_scale_max_form(yrow, N, k, stride, s, 0);
 }
 
 /* The linear part for a list of rows: y[r*N + n] for r < nrows. */
@@ -118,13 +142,14 @@ void orc_linear_rows(const float* x, const float* W, const float* b,
 /*
  * The whole path for a list of rows.  out has nrows*N floats for kinds (a),
  * (b) and none, and nrows floats for (c).  y_scratch, when not NULL, must hold
- * nrows*N doubles and receives the linear outputs.  Returns 0, or -1 on a
- * shape/argument error (no windows for (c), unknown kind, bad row index).
+ * nrows*N doubles and receives the linear outputs.  gelu_tanh selects the
+ * tanh form of GELU for (a) and (c).  Returns 0, or -1 on a shape/argument
+ * error (no windows for (c), unknown kind, bad row index).
  */
 int orc_forward_rows(const float* x, const float* W, const float* b,
                      int64_t M, int64_t K, int64_t N, int kind,
                      double scale, double clamp_lo, double clamp_hi,
-                     int64_t pool_k, int64_t pool_stride,
+                     int64_t pool_k, int64_t pool_stride, int gelu_tanh,
                      const int64_t* rows, int64_t nrows,
                      float* out, double* y_scratch) {
     if (M < 0 || K < 0 || N <= 0 || nrows < 0) return -1;
@@ -146,13 +171,13 @@ int orc_forward_rows(const float* x, const float* W, const float* b,
     for (int64_t r = 0; r < nrows; ++r) {
         const double* yr = y + r * N;
         if (kind == ORC_EPI_AVGPOOL_GELU_SCALE_ROWMAX) {
-            out[r] = (float)orc_pool_gelu_scale_max(yr, N, pool_k, pool_stride, scale);
+            out[r] = (float)orc_pool_gelu_scale_max_form(yr, N, pool_k, pool_stride, scale, gelu_tanh);
             continue;
         }
         for (int64_t n = 0; n < N; ++n) {
             double o;
             if (kind == ORC_EPI_SCALE_HARDTANH_GELU)
-                o = orc_scale_hardtanh_gelu(yr[n], scale, clamp_lo, clamp_hi);
+                o = orc_scale_hardtanh_gelu_form(yr[n], scale, clamp_lo, clamp_hi, gelu_tanh);
             else if (kind == ORC_EPI_SWISH_SCALE)
                 o = orc_swish_scale(yr[n], scale);
             else

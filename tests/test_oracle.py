@@ -145,6 +145,56 @@ def test_gelu_is_erf_form_not_tanh_form():
 # Epilogue (a): scale -> hardtanh -> GELU
 # --------------------------------------------------------------------------
 
+def test_gelu_tanh_form_closed_forms():
+    # The tanh form (page l2_p53's first fused kernel): v/2 (1 + tanh(c (v +
+    # 0.044715 v^3))), c = sqrt(2/pi).  tanh is odd, so the same identity as
+    # the erf form holds: G(v) - G(-v) = v; G(0) = 0; G(v) -> v and -> 0.
+    assert oracle.gelu_tanh(0.0) == 0.0
+    for v in [0.1, 0.75, 1.0, 1.7, 2.0, 3.3]:
+        assert abs((oracle.gelu_tanh(v) - oracle.gelu_tanh(-v)) - v) < 1e-15
+    assert abs(oracle.gelu_tanh(30.0) - 30.0) < 1e-12
+    assert abs(oracle.gelu_tanh(-30.0)) < 1e-12
+    # curvature at 0: G(h) + G(-h) = h tanh(c (h + 0.044715 h^3)) ~ c h^2,
+    # which pins c = sqrt(2/pi) = 0.7978845608...
+    h = 1e-4
+    assert abs((oracle.gelu_tanh(h) + oracle.gelu_tanh(-h)) / h**2 - 0.7978845608) < 1e-6
+
+
+def test_gelu_tanh_form_distance_from_erf_form():
+    # Against the (independently pinned) erf form: the approximation is off
+    # by at most 4.73e-4, at |v| ~ 2.70, and by 9.80e-5 at v = 2 (the page's
+    # printed figure for that gap is garbled; these are the values of the two
+    # closed forms).  A wrong constant or a dropped factor moves both (e.g.
+    # 0.04715 for 0.044715 gives a 1.5e-3 gap).
+    xs = np.linspace(-8, 8, 16001)
+    d = np.array([oracle.gelu_tanh(v) - oracle.gelu(v) for v in xs])
+    i = int(np.abs(d).argmax())
+    assert 4.6e-4 < abs(d[i]) < 4.8e-4
+    assert 2.6 < abs(xs[i]) < 2.8
+    assert abs((oracle.gelu_tanh(2.0) - oracle.gelu(2.0)) - 9.80e-5) < 1e-6
+    # the gap is even in v (both forms satisfy G(v) - G(-v) = v)
+    assert np.allclose(d, d[::-1], rtol=0, atol=1e-13)
+
+
+def test_forward_with_tanh_form():
+    # gelu_tanh switches the GELU of epilogues (a) and (c), nothing else
+    x = np.array([[1.0, -2.0, 0.5, 3.0]], dtype=np.float32)
+    W = np.array([[0.5, 0.25, -1.0, 0.125], [1.0, 1.0, 1.0, 1.0]], dtype=np.float32)
+    b = np.array([0.25, -0.5], dtype=np.float32)
+    y = oracle.linear_rows(x, W, b)[0]
+    a = oracle.forward_rows(x, W, b, gelu_tanh=True, **oracle.PROBLEMS["scale_hardtanh_gelu"])[0]
+    for n in range(2):
+        t = min(max(0.5 * y[n], -2.0), 2.0)
+        assert a[n] == np.float32(oracle.gelu_tanh(t))
+    sw = oracle.forward_rows(x, W, b, gelu_tanh=True, **oracle.PROBLEMS["swish_scale"])
+    assert (sw == oracle.forward_rows(x, W, b, **oracle.PROBLEMS["swish_scale"])).all()
+    Wp = np.tile(W, (8, 1))  # N = 16: one pool window
+    bp = np.tile(b, 8)
+    c = oracle.forward_rows(x, Wp, bp, gelu_tanh=True, **oracle.PROBLEMS["avgpool_gelu_scale_rowmax"])[0]
+    p = oracle.linear_rows(x, Wp, bp)[0].mean()
+    assert c == np.float32(2.0 * oracle.gelu_tanh(p))
+
+
 def test_epilogue_a_saturation_and_order(normal_values):
     tb = {e["quantity"]: e["value"] for e in normal_values["textbook_values"]}
     f = oracle.scale_hardtanh_gelu
