@@ -41,6 +41,8 @@ CONFIGS = {
     "sweep_m256_k8192_n8192_hardtanh_gelu": (256, 8192, 8192, "scale_hardtanh_gelu"),
     "sweep_m1024_k8192_n8192_hardtanh_gelu": (1024, 8192, 8192, "scale_hardtanh_gelu"),
     "sweep_m4096_k8192_n8192_hardtanh_gelu": (4096, 8192, 8192, "scale_hardtanh_gelu"),
+    # the Linear alone (bias, no epilogue): the pages' addmm comparator
+    "linear2048x8192x8192_bias_only": (2048, 8192, 8192, "none"),
     # epilogue (c) by pooled weights: pool W and b every call, or reuse them
     "poolfold_per_call_1024x8192x8192_pool16_gelu_rowmax": (1024, 8192, 8192, "avgpool_gelu_scale_rowmax"),
     "poolfold_cached_1024x8192x8192_pool16_gelu_rowmax": (1024, 8192, 8192, "avgpool_gelu_scale_rowmax"),

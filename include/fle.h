@@ -57,11 +57,27 @@ typedef enum {
     FLE_PREC_TF32 = 1
 } fle_precision;
 
+/* Options (fle_epilogue_desc.flags, bitwise or; 0 is the pages' problems).
+ * FLE_FLAG_GELU_TANH: (a), (c) use GELU in its tanh form,
+ *   v/2 * (1 + tanh(sqrt(2/pi) * (v + 0.044715 v^3))), the approximation page
+ *   "Kimi-K2.6 l2_p53" writes into its first fused elementwise kernel before
+ *   choosing the exact erf form (the default here).
+ * FLE_FLAG_FOLD_SCALE: (a) applies the scale as s*acc + s*b in one fused
+ *   multiply-add, the pages' idea of folding the constant into the GEMM's
+ *   alpha (page "Kimi-K2.6 l2_p53", its cuBLAS alpha/beta discussion).  The
+ *   same function; only the fp32 rounding of that step differs.  Ignored by
+ *   the other kinds, whose scale comes after a nonlinearity. */
+enum {
+    FLE_FLAG_GELU_TANH = 1,
+    FLE_FLAG_FOLD_SCALE = 2
+};
+
 /* Parameters of the epilogue.  Fields that a kind does not use are ignored.
  *   scale              (a), (b), (c): multiplier
  *   clamp_lo, clamp_hi (a): Hardtanh bounds, clamp_lo <= clamp_hi
  *   pool_k, pool_stride(c): window and stride; this build supports
- *                       pool_stride == pool_k with pool_k in {1,2,4,8,16,32} */
+ *                       pool_stride == pool_k with pool_k in {1,2,4,8,16,32}
+ *   flags              FLE_FLAG_* options; unknown bits are FLE_ERR_DESC */
 typedef struct {
     int32_t kind;
     int32_t precision;
@@ -70,6 +86,7 @@ typedef struct {
     float clamp_hi;
     int32_t pool_k;
     int32_t pool_stride;
+    int32_t flags;
 } fle_epilogue_desc;
 
 /* Status codes. */
@@ -79,8 +96,8 @@ enum {
     FLE_ERR_SHAPE = 2,       /* negative size, size >= 2^31, or (c) N < pool_k */
     FLE_ERR_ALIGN = 3,       /* x or W not 16-byte aligned, K % 4 != 0, or
                                 out / b not 4-byte aligned                   */
-    FLE_ERR_DESC = 4,        /* unknown kind/precision, non-finite scale or
-                                clamp, clamp_lo > clamp_hi, unsupported pool  */
+    FLE_ERR_DESC = 4,        /* unknown kind/precision/flag, non-finite scale
+                                or clamp, clamp_lo > clamp_hi, unsupported pool */
     FLE_ERR_WORKSPACE = 5,   /* workspace smaller than fle_workspace_size()  */
     FLE_ERR_ARCH = 6,        /* current device is not sm_100 (B200)          */
     FLE_ERR_CUDA = 7,        /* a CUDA runtime/driver call failed            */
@@ -236,10 +253,11 @@ int fle_test_bounded_wait(uint32_t timeout_us, void* stream);
 
 /*
  * Test hook for the epilogue's scalar math: out[i] = f(in[i]) for device
- * arrays of n floats, with f = erf (which = 0), exact-form GELU (1) or
- * x * sigmoid(x) (2), evaluated either as the fused epilogue evaluates it
- * (reference = 0) or with CUDA's erff/expf and IEEE division (reference = 1),
- * so tests can bound the difference.  Stream-ordered.
+ * arrays of n floats, with f = erf (which = 0), exact-form GELU (1),
+ * x * sigmoid(x) (2) or tanh-form GELU (3), evaluated either as the fused
+ * epilogue evaluates it (reference = 0) or with CUDA's erff/expf/tanhf and
+ * IEEE division (reference = 1), so tests can bound the difference.
+ * Stream-ordered.
  */
 int fle_test_epilogue_math(const float* in, float* out, int64_t n, int32_t which, int32_t reference,
                            void* stream);

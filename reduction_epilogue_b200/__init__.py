@@ -31,6 +31,8 @@ EPI_AVGPOOL_GELU_SCALE_ROWMAX = 2
 EPI_NONE = 3
 PREC_3XTF32 = 0
 PREC_TF32 = 1
+FLAG_GELU_TANH = 1
+FLAG_FOLD_SCALE = 2
 
 FLE_OK = 0
 STATUS_NAMES = {
@@ -57,6 +59,7 @@ class EpilogueDesc(ctypes.Structure):
         ("clamp_hi", ctypes.c_float),
         ("pool_k", ctypes.c_int32),
         ("pool_stride", ctypes.c_int32),
+        ("flags", ctypes.c_int32),
     ]
 
 
@@ -118,17 +121,23 @@ def _status_text(status: int) -> str:
         return "?"
 
 
-def desc_for(problem: str | None = None, precision: str | int = "tf32", **overrides) -> EpilogueDesc:
-    """Builds an EpilogueDesc from a page problem name and/or explicit fields."""
+def desc_for(problem: str | None = None, precision: str | int = "tf32", gelu: str = "erf",
+             fold_scale: bool = False, **overrides) -> EpilogueDesc:
+    """Builds an EpilogueDesc from a page problem name and/or explicit fields.
+    gelu="tanh" selects FLE_FLAG_GELU_TANH; fold_scale selects
+    FLE_FLAG_FOLD_SCALE."""
     f = dict(kind=EPI_NONE, scale=1.0, clamp_lo=-2.0, clamp_hi=2.0, pool_k=16)
     if problem is not None:
         f.update(PROBLEMS[problem])
     f.update(overrides)
     if isinstance(precision, str):
         precision = {"tf32": PREC_TF32, "3xtf32": PREC_3XTF32}[precision.lower()]
+    if gelu not in ("erf", "tanh"):
+        raise ValueError("gelu must be 'erf' or 'tanh'")
+    flags = int(f.get("flags", 0)) | (FLAG_GELU_TANH if gelu == "tanh" else 0) | (FLAG_FOLD_SCALE if fold_scale else 0)
     pk = int(f["pool_k"])
     return EpilogueDesc(int(f["kind"]), int(precision), float(f["scale"]), float(f["clamp_lo"]),
-                        float(f["clamp_hi"]), pk, int(f.get("pool_stride", pk)))
+                        float(f["clamp_hi"]), pk, int(f.get("pool_stride", pk)), flags)
 
 
 def _ptr(t) -> int | None:

@@ -122,6 +122,7 @@ int check_desc(const fle_epilogue_desc* d) {
     if (!d) return FLE_ERR_NULL;
     if (d->kind < FLE_EPI_SCALE_HARDTANH_GELU || d->kind > FLE_EPI_NONE) return FLE_ERR_DESC;
     if (d->precision != FLE_PREC_3XTF32 && d->precision != FLE_PREC_TF32) return FLE_ERR_DESC;
+    if (d->flags & ~(FLE_FLAG_GELU_TANH | FLE_FLAG_FOLD_SCALE)) return FLE_ERR_DESC;
     if (d->kind != FLE_EPI_NONE && !std::isfinite(d->scale)) return FLE_ERR_DESC;
     if (d->kind == FLE_EPI_SCALE_HARDTANH_GELU) {
         if (!std::isfinite(d->clamp_lo) || !std::isfinite(d->clamp_hi) || d->clamp_lo > d->clamp_hi)
@@ -512,6 +513,8 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
     p.scale = d->scale;
     p.clamp_lo = d->clamp_lo;
     p.clamp_hi = d->clamp_hi;
+    p.gelu_tanh = (d->flags & FLE_FLAG_GELU_TANH) ? 1 : 0;
+    p.fold_scale = (d->flags & FLE_FLAG_FOLD_SCALE) ? 1 : 0;
     p.pool_k = pool ? d->pool_k : 1;
     p.pool_limit = pool ? (N / d->pool_k) * d->pool_k : N;
     p.vec_out = ((reinterpret_cast<uintptr_t>(out) & 15u) == 0 && N % 4 == 0) ? 1 : 0;
@@ -711,7 +714,7 @@ int fle_device_status(void* stream) {
 int fle_test_epilogue_math(const float* in, float* out, int64_t n, int32_t which, int32_t reference,
                            void* stream) {
     if (!in || !out) return FLE_ERR_NULL;
-    if (n < 0 || which < 0 || which > 2) return FLE_ERR_SHAPE;
+    if (n < 0 || which < 0 || which > 3) return FLE_ERR_SHAPE;
     DeviceInfo di;
     int st = device_info(&di);
     if (st != FLE_OK) return st;

@@ -68,6 +68,8 @@ struct KParams {
     int sk_grid;            // CTAs [0, sk_grid) share the stream-K k-blocks
     int kind;
     float scale, clamp_lo, clamp_hi;
+    int gelu_tanh;          // GELU in its tanh form, (a) and (c)
+    int fold_scale;         // (a): scale * acc + scale * b in one FMA
     int pool_k;
     int64_t pool_limit;     // columns covered by complete pool windows
     int vec_out;            // out 16-byte aligned and N % 4 == 0
@@ -199,12 +201,25 @@ __device__ __forceinline__ float gelu_erf(float t) {
     return t * 0.5f * (1.0f + erf_as7126(t * 0.70710678118654752440f));
 }
 
+// GELU in its tanh form, t/2 * (1 + tanh(u)), u = sqrt(2/pi) (t + 0.044715 t^3),
+// with tanh(u) = 1 - 2 / (1 + e^(2u)): one exponential and one division; it
+// saturates to +-1 where e^(2u) over- or underflows.
+__device__ __forceinline__ float gelu_tanh_form(float t) {
+    const float u = 0.79788456080286535588f * fmaf(0.044715f * t, t * t, t);
+    const float th = 1.0f - __fdividef(2.0f, 1.0f + __expf(2.0f * u));
+    return 0.5f * t * (1.0f + th);
+}
+
+__device__ __forceinline__ float gelu_sel(float t, const KParams& p) {
+    return p.gelu_tanh ? gelu_tanh_form(t) : gelu_erf(t);
+}
+
 template <int KIND>
 __device__ __forceinline__ float epi_apply(float y, const KParams& p) {
     if constexpr (KIND == kEpiHardtanhGelu) {
-        float t = y * p.scale;
+        float t = p.fold_scale ? y : y * p.scale;  // folded: y already holds s*acc + s*b
         t = fminf(fmaxf(t, p.clamp_lo), p.clamp_hi);
-        return gelu_erf(t);
+        return gelu_sel(t, p);
     } else if constexpr (KIND == kEpiSwish) {
         // y * sigmoid(y); for y -> -inf, exp(-y) overflows to inf and the
         // quotient goes to 0 (the limit), never NaN.
@@ -223,6 +238,16 @@ __device__ __forceinline__ void atomic_max_f32(float* addr, float v) {
         atomicMax(reinterpret_cast<int*>(addr), __float_as_int(v));
     else
         atomicMin(reinterpret_cast<unsigned*>(addr), __float_as_uint(v));
+}
+
+// v[j] = s * v[j] + s * b[n0 + j] in one FMA: (a) with the scale folded in.
+__device__ __forceinline__ void fold_bias32(const KParams& p, int64_t n0, float (&v)[32]) {
+    const float s = p.scale;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const float bj = (p.bias != nullptr && n0 + j < p.N) ? __ldg(p.bias + n0 + j) : 0.0f;
+        v[j] = fmaf(s, v[j], s * bj);
+    }
 }
 
 // v[j] += b[n0 + j] for the columns that exist, four at a time (no extra
@@ -257,7 +282,10 @@ struct EpiOut {
 template <int KIND>
 __device__ __forceinline__ void epi_store_direct(const KParams& p, const EpiOut& eo, int64_t m, int64_t n0,
                                                  float (&v)[32]) {
-    add_bias32(p, n0, v);
+    if (KIND == kEpiHardtanhGelu && p.fold_scale)
+        fold_bias32(p, n0, v);
+    else
+        add_bias32(p, n0, v);
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = epi_apply<KIND>(v[j], p);
     if (eo.tmap != nullptr) {
@@ -304,7 +332,7 @@ __device__ __forceinline__ void epi_pool_direct(const KParams& p, int64_t n0, fl
         acc += v[j];
         if (((j + 1) & (k - 1)) == 0) {
             if (n0 + j + 1 <= p.pool_limit) {
-                float g = p.scale * gelu_erf(acc * inv_k);
+                float g = p.scale * gelu_sel(acc * inv_k, p);
                 best = fmaxf(best, g);
             }
             acc = 0.0f;
@@ -317,9 +345,11 @@ template <int KIND>
 __device__ __forceinline__ void epi_store_swapped(const KParams& p, int64_t n, int64_t m0, float (&v)[32]) {
     const float bn = (p.bias != nullptr && n < p.N) ? __ldg(p.bias + n) : 0.0f;
     const bool n_ok = n < p.N;
+    const bool fold = KIND == kEpiHardtanhGelu && p.fold_scale;
+    const float sbn = p.scale * bn;
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
-        const float o = epi_apply<KIND>(v[j] + bn, p);
+        const float o = epi_apply<KIND>(fold ? fmaf(p.scale, v[j], sbn) : v[j] + bn, p);
         if (n_ok && m0 + j < p.M) p.out[(m0 + j) * p.N + n] = o;
     }
 }
@@ -831,7 +861,7 @@ __global__ void fle_bias_only_kernel(const KParams p) {
         for (int64_t w0 = 0; w0 + p.pool_k <= p.pool_limit; w0 += p.pool_k) {
             float acc = 0.0f;
             for (int t = 0; t < p.pool_k; ++t) acc += p.bias ? p.bias[w0 + t] : 0.0f;
-            best = fmaxf(best, p.scale * gelu_erf(acc / static_cast<float>(p.pool_k)));
+            best = fmaxf(best, p.scale * gelu_sel(acc / static_cast<float>(p.pool_k), p));
         }
         p.out[i] = best;
         return;
@@ -840,7 +870,7 @@ __global__ void fle_bias_only_kernel(const KParams p) {
     const float y = p.bias ? p.bias[i % p.N] : 0.0f;
     float o;
     switch (p.kind) {
-        case kEpiHardtanhGelu: o = epi_apply<kEpiHardtanhGelu>(y, p); break;
+        case kEpiHardtanhGelu: o = epi_apply<kEpiHardtanhGelu>(p.fold_scale ? p.scale * y : y, p); break;
         case kEpiSwish: o = epi_apply<kEpiSwish>(y, p); break;
         default: o = y; break;
     }
@@ -890,14 +920,16 @@ __global__ void fle_pool_weights_kernel(const float* __restrict__ W, const float
 }
 
 // Test hook: the epilogue's scalar functions on n inputs (kind 0: erf,
-// 1: GELU, 2: swish with scale 1), for checks against CUDA's erff/expf.
+// 1: GELU, 2: swish with scale 1, 3: GELU in its tanh form), for checks
+// against CUDA's erff / expf / tanhf.
 __global__ void fle_math_probe_kernel(const float* in, float* out, int64_t n, int which) {
     const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i >= n) return;
     const float v = in[i];
     if (which == 0) out[i] = erf_as7126(v);
     else if (which == 1) out[i] = gelu_erf(v);
-    else out[i] = __fdividef(v, 1.0f + __expf(-v));
+    else if (which == 2) out[i] = __fdividef(v, 1.0f + __expf(-v));
+    else out[i] = gelu_tanh_form(v);
 }
 __global__ void fle_math_reference_kernel(const float* in, float* out, int64_t n, int which) {
     const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -905,7 +937,8 @@ __global__ void fle_math_reference_kernel(const float* in, float* out, int64_t n
     const float v = in[i];
     if (which == 0) out[i] = erff(v);
     else if (which == 1) out[i] = v * 0.5f * (1.0f + erff(v * 0.70710678118654752440f));
-    else out[i] = v / (1.0f + expf(-v));
+    else if (which == 2) out[i] = v / (1.0f + expf(-v));
+    else out[i] = 0.5f * v * (1.0f + tanhf(0.79788456080286535588f * (v + 0.044715f * v * v * v)));
 }
 
 // Test hook: one thread waits on a barrier nothing arrives on.

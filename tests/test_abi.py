@@ -73,6 +73,13 @@ def test_null_and_descriptor_errors(lib):
     assert _call(lib, 4, 8, 64, bad) == 4
     bad = fle.desc_for("avgpool_gelu_scale_rowmax"); bad.pool_stride = 8
     assert _call(lib, 4, 8, 64, bad) == 4
+    bad = fle.desc_for("scale_hardtanh_gelu"); bad.flags = 4  # unknown option bit
+    assert _call(lib, 4, 8, 8, bad) == 4
+    # the option bits mirror include/fle.h
+    ok = fle.desc_for("scale_hardtanh_gelu", gelu="tanh", fold_scale=True)
+    assert ok.flags == fle.FLAG_GELU_TANH | fle.FLAG_FOLD_SCALE == 3
+    with pytest.raises(ValueError):
+        fle.desc_for("scale_hardtanh_gelu", gelu="sigmoid")
 
 
 def test_shape_and_alignment_errors(lib):

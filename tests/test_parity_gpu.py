@@ -276,7 +276,7 @@ def test_long_k_accuracy_3xtf32(fle, precision):
         _assert_close(out.cpu().numpy()[rows], _oracle(x, W, b, "none", rows=rows), precision, f"K=32768 {M}x{N}")
 
 
-@pytest.mark.parametrize("which", [0, 1, 2])
+@pytest.mark.parametrize("which", [0, 1, 2, 3])
 def test_epilogue_math_against_fp64_and_cuda(fle, which):
     # The epilogue evaluates erf by Abramowitz & Stegun 7.1.26 (|error| <=
     # 1.5e-7) and the sigmoid with a fast exponential and divide; bound both
@@ -303,9 +303,13 @@ def test_epilogue_math_against_fp64_and_cuda(fle, which):
     elif which == 1:
         exact = x * 0.5 * (1 + erf64(x / np.sqrt(2)))
         bound = 2.5e-7 * np.maximum(1.0, np.abs(x))
-    else:
-        exact = x / (1 + np.exp(-x))
+    elif which == 2:
+        with np.errstate(over="ignore"):
+            exact = x / (1 + np.exp(-x))
         bound = 4e-6 * np.maximum(1.0, np.abs(x))
+    else:
+        exact = 0.5 * x * (1 + np.tanh(np.sqrt(2 / np.pi) * (x + 0.044715 * x ** 3)))
+        bound = 5e-7 * np.maximum(1.0, np.abs(x))
     assert np.isfinite(g).all()
     assert np.abs(g - exact).max() <= bound.max() and (np.abs(g - exact) <= bound).all()
     assert (np.abs(g - c) <= 2 * bound).all()
@@ -368,3 +372,48 @@ def test_swapped_pair_tiles(fle, M, problem):
     x, W, b = synth.linear_inputs(M, K, N, seed=11, device="cuda")
     out = _run(fle, x, W, b, problem, "tf32")
     _assert_close(out.cpu().numpy(), _oracle(x, W, b, problem), "tf32", f"{M}x{K}x{N} {plan}")
+
+
+OPTION_SHAPES = [(7, 36, 33), (100, 1056, 520), (200, 64, 301), (300, 132, 1000), (128, 520, 19107)]
+
+
+@pytest.mark.parametrize("precision", ["tf32", "3xtf32"])
+@pytest.mark.parametrize("problem", ["scale_hardtanh_gelu", "avgpool_gelu_scale_rowmax"])
+@pytest.mark.parametrize("M,K,N", OPTION_SHAPES)
+def test_gelu_tanh_option(fle, M, K, N, problem, precision):
+    # FLE_FLAG_GELU_TANH: the tanh form of GELU in (a) and (c), against the
+    # oracle's tanh form (the swapped, direct and swapped-pair kernels).
+    if problem == "avgpool_gelu_scale_rowmax" and N < 16:
+        pytest.skip("pool needs N >= 16")
+    x, W, b = synth.linear_inputs(M, K, N, seed=3 * M + K + N, device="cuda")
+    out = fle.linear_epilogue(x, W, b, problem, precision, gelu="tanh")
+    torch.cuda.synchronize()
+    assert fle.device_status() == 0
+    ref = oracle.forward_rows(x.cpu().numpy(), W.cpu().numpy(), b.cpu().numpy(), gelu_tanh=True,
+                              **oracle.PROBLEMS[problem])
+    _assert_close(out.cpu().numpy(), ref, precision, f"tanh GELU {problem} {M}x{K}x{N}")
+    # and it is not the erf form: the two differ by up to 4.7e-4 per element
+    if problem == "scale_hardtanh_gelu":
+        erf_ref = _oracle(x, W, b, problem)
+        assert np.abs(ref.astype(np.float64) - erf_ref).max() > 1e-6
+
+
+@pytest.mark.parametrize("precision", ["tf32", "3xtf32"])
+@pytest.mark.parametrize("M,K,N", OPTION_SHAPES)
+def test_fold_scale_option(fle, M, K, N, precision):
+    # FLE_FLAG_FOLD_SCALE: (a) as s*acc + s*b in one FMA; the same function,
+    # so the same oracle and tolerance; and the saturated region too.
+    x, W, b = synth.linear_inputs(M, K, N, seed=5 * M + K + N, device="cuda")
+    x50 = x * 50.0
+    for xin in (x, x50):
+        out = fle.linear_epilogue(xin, W, b, "scale_hardtanh_gelu", precision, fold_scale=True)
+        torch.cuda.synchronize()
+        assert fle.device_status() == 0
+        ref = _oracle(xin, W, b, "scale_hardtanh_gelu")
+        if xin is x:
+            _assert_close(out.cpu().numpy(), ref, precision, f"fold scale {M}x{K}x{N}")
+        else:
+            # TF32 operand error grows with |x| (x 50): scale the bound likewise
+            atol, rtol = TOL[precision]
+            err = np.abs(out.cpu().numpy().astype(np.float64) - ref)
+            assert (err <= 50 * (atol + rtol * np.abs(ref))).all()
