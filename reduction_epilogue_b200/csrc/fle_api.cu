@@ -253,11 +253,20 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
     const bool force_dp = std::strcmp(ov, "dp") == 0;
     const bool force_sk = std::strcmp(ov, "sk") == 0;
     // the stream-K minimum is 16 k-blocks of 32 (512 of K) per CTA
-    const int64_t min_iters = kMinSkIters * fle::kBK / pl.bk;
+    // (FLE_MIN_KB overrides it for comparisons)
+    static const int64_t min_kb_env = [] {
+        const char* e = std::getenv("FLE_MIN_KB");
+        const long v = e ? std::atol(e) : 0;
+        return static_cast<int64_t>(v > 0 ? v : 0);
+    }();
+    const int64_t min_iters = min_kb_env > 0 ? min_kb_env : kMinSkIters * fle::kBK / pl.bk;
     pl.dp_tiles = static_cast<int>(T);
     pl.grid = static_cast<int>(T < G ? T : G);
     pl.sk_grid = 0;
-    if (!force_dp && T % G != 0 && pl.num_kb >= 2 * min_iters) {
+    // Splitting K costs a partial-tile round trip and a wait at the end of the
+    // tile (a few microseconds); it is taken only for tiles of at least four
+    // minimum-size parts (measured: at K = 1024 the whole tiles are faster).
+    if (!force_dp && T % G != 0 && pl.num_kb >= 4 * min_iters) {
         if (force_sk) {
             // spread all k-blocks evenly over all SMs (measured no faster
             // than the k-aligned split below on any of the benchmark shapes,

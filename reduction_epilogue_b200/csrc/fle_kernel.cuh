@@ -50,7 +50,7 @@ enum : int { kPrec3xTF32 = 0, kPrecTF32 = 1 };
 // Wait-site identifiers recorded with a timeout.
 enum : unsigned {
     kWhereProdEmpty = 1, kWhereMmaFull = 2, kWhereMmaAccEmpty = 3, kWhereEpiAccFull = 4,
-    kWhereConvFull = 5, kWhereDrain = 6, kWhereProdDrain = 7, kWhereFixup = 8, kWhereTest = 9
+    kWhereConvFull = 5, kWhereDrain = 6, kWhereProdDrain = 7, kWhereTest = 9
 };
 
 struct KParams {
@@ -392,29 +392,12 @@ __device__ __forceinline__ void epi_finish(const KParams& p, const Unit& u, int 
     __syncwarp();
 }
 
-// Waits until *counter >= target (other CTAs raise it with atomicAdd after
-// a __threadfence), reading it with acquire semantics.  Bounded like the
-// mbarrier waits: gives up on *abort or after timeout_ns (recording a
-// timeout at `where` and raising *abort).
-__device__ __forceinline__ bool wait_count_bounded(const unsigned* counter, unsigned target, volatile int* abort,
-                                                   uint64_t timeout_ns, unsigned where) {
-    uint64_t t0 = 0;
-    uint32_t spins = 0;
-    while (true) {
-        unsigned v;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
-        if (v >= target) return true;
-        if (*abort) return false;
-        if (t0 == 0) t0 = global_timer_ns();
-        if ((++spins & 15u) == 0u) {
-            if (global_timer_ns() - t0 > timeout_ns) {
-                record_error(8u, where);
-                *abort = 1;
-                return false;
-            }
-            __nanosleep(100);
-        }
-    }
+// A global word read with acquire semantics (stream-K arrival counters,
+// raised by other CTAs with atomicAdd after a __threadfence).
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
 
 // Barrier among the eight epilogue warps only (named barrier 1, 256 threads).
@@ -737,12 +720,34 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 #undef FLE_EPI_BODY
                 epi_finish<SWAP>(p, u, r, best);
                 if constexpr (!kRegAcc) release_acc();
-            } else if (u.kb0 != 0) {
-                // Not the tile's finisher: park this CTA's fp32 partial tile in
-                // its workspace slot, column-major inside the tile (element
-                // (row, col) at col * 128 + row) so that a warp's lanes write
-                // 32 consecutive floats, then count it on the tile's counter.
-                float* slot = p.ws + static_cast<size_t>(2 * blockIdx.x + u.slot) * kBM * BN;
+            } else {
+                // A unit of a tile whose k-blocks are split over CTAs first ..
+                // last.  The CTA holding k-block 0 (the last unit of its range,
+                // while the others ran the tile's later k-blocks as their first
+                // units) normally ends last: if every other contributor has
+                // already parked its partial, it adds them to its own
+                // accumulator and runs the epilogue.  Otherwise it parks its
+                // partial too, and whichever contributor arrives last sums all
+                // partials.  No CTA ever waits for another.  Partials are summed
+                // in CTA order (= k order), so the result does not depend on
+                // who does it.
+                const int64_t tsk = u.sk_tile;
+                const int first = sk_cta_of(tsk * p.num_kb, p.sk_iters, p.sk_grid);
+                const int last = sk_cta_of((tsk + 1) * p.num_kb - 1, p.sk_iters, p.sk_grid);
+                const unsigned others = static_cast<unsigned>(last - first);
+                unsigned* counter = p.counters + tsk;
+                if (u.kb0 == 0) {
+                    if (threadIdx.x == 128) *last_flag = (ld_acquire_u32(counter) == others) ? 1 : 0;
+                    __syncwarp();  // named barriers are .aligned: whole warps arrive
+                    epilogue_bar_sync();
+                }
+                const bool own = (u.kb0 == 0) && *last_flag != 0;
+                bool fix = own;
+                if (!own) {
+                    // park the partial, column-major inside the tile (element
+                    // (row, col) at col * 128 + row: a warp's lanes write 32
+                    // consecutive floats), then count it
+                    float* slot = p.ws + static_cast<size_t>(2 * blockIdx.x + u.slot) * kBM * BN;
 #define FLE_PARK_BODY(lc)                                                                 \
     {                                                                                     \
         float v[32];                                                                      \
@@ -750,52 +755,44 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         float* d = slot + static_cast<size_t>((c_lo + (lc)) * 32) * kBM + r;              \
         _Pragma("unroll") for (int j = 0; j < 32; ++j) __stcg(d + j * kBM, v[j]);         \
     }
-                if constexpr (kRegAcc) {
+                    if constexpr (kRegAcc) {
 #pragma unroll
-                    for (int lc = 0; lc < kHalf; ++lc)
-                        if (lc < mine) FLE_PARK_BODY(lc)
-                } else {
+                        for (int lc = 0; lc < kHalf; ++lc)
+                            if (lc < mine) FLE_PARK_BODY(lc)
+                    } else {
 #pragma unroll 1
-                    for (int lc = 0; lc < mine; ++lc) FLE_PARK_BODY(lc)
-                }
+                        for (int lc = 0; lc < mine; ++lc) FLE_PARK_BODY(lc)
+                    }
 #undef FLE_PARK_BODY
-                if constexpr (!kRegAcc) release_acc();
-                __threadfence();
-                epilogue_bar_sync();
-                if (threadIdx.x == 128) atomicAdd(p.counters + u.sk_tile, 1u);
-                __syncwarp();
-            } else {
-                // The tile's finisher: this unit holds k-block 0, the last unit
-                // of this CTA (its range ends inside the tile), while the other
-                // contributors ran the tile's later k-blocks as their first
-                // units.  Wait until all of them have parked their partials,
-                // then add them to this CTA's own accumulator in CTA order
-                // (= k order: a fixed order, so results are reproducible) and
-                // run the epilogue on the sum.
-                const int64_t tsk = u.sk_tile;
-                const int first = static_cast<int>(blockIdx.x);
-                const int last = sk_cta_of((tsk + 1) * p.num_kb - 1, p.sk_iters, p.sk_grid);
-                if (threadIdx.x == 128)
-                    *last_flag = wait_count_bounded(p.counters + tsk, static_cast<unsigned>(last - first),
-                                                    abort_flag, p.timeout_ns, kWhereFixup)
-                                     ? 1 : 0;
-                __syncwarp();  // named barriers are .aligned: whole warps arrive
-                epilogue_bar_sync();
-                const bool have = *last_flag != 0;
-                __threadfence();
-                float best = -INFINITY;
-                auto src_of = [&](int cc, int c) {
-                    const int sl = sk_slot_of(cc, tsk, p.sk_iters, p.sk_grid, p.num_kb);
-                    return p.ws + static_cast<size_t>(2 * cc + sl) * kBM * BN + static_cast<size_t>(c * 32) * kBM + r;
-                };
-                // own accumulator, then contributors first+1 .. last; loads of
-                // up to three contributors are in flight together
+                    if constexpr (!kRegAcc) release_acc();
+                    __threadfence();
+                    epilogue_bar_sync();
+                    if (threadIdx.x == 128) *last_flag = (atomicAdd(counter, 1u) == others) ? 1 : 0;
+                    __syncwarp();
+                    epilogue_bar_sync();
+                    fix = *last_flag != 0;
+                }
+                if (fix) {
+                    __threadfence();
+                    float best = -INFINITY;
+                    auto src_of = [&](int cc, int c) {
+                        const int sl = sk_slot_of(cc, tsk, p.sk_iters, p.sk_grid, p.num_kb);
+                        return p.ws + static_cast<size_t>(2 * cc + sl) * kBM * BN +
+                               static_cast<size_t>(c * 32) * kBM + r;
+                    };
+                    // start from the own accumulator (contributors first+1 ..
+                    // last to add) or from zero (first .. last); loads of up to
+                    // three contributors are in flight together
 #define FLE_FIX_BODY(lc)                                                                      \
     {                                                                                         \
         const int c = c_lo + (lc);                                                            \
         float v[32];                                                                          \
-        FLE_LOAD_ACC(lc, v);                                                                  \
-        int cc = first + 1;                                                                   \
+        if (own) {                                                                            \
+            FLE_LOAD_ACC(lc, v);                                                              \
+        } else {                                                                              \
+            _Pragma("unroll") for (int j = 0; j < 32; ++j) v[j] = 0.0f;                       \
+        }                                                                                     \
+        int cc = own ? first + 1 : first;                                                     \
         for (; cc + 2 <= last; cc += 3) {                                                     \
             const float* s0 = src_of(cc, c);                                                  \
             const float* s1 = src_of(cc + 1, c);                                              \
@@ -816,7 +813,6 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         }                                                                                     \
         epi_chunk<SWAP, BN>(p, u, r, c, v, best, eo);                                         \
     }
-                if (have) {
                     if constexpr (kRegAcc) {
 #pragma unroll
                         for (int lc = 0; lc < kHalf; ++lc)
@@ -825,13 +821,14 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 #pragma unroll 1
                         for (int lc = 0; lc < mine; ++lc) FLE_FIX_BODY(lc)
                     }
-                    epi_finish<SWAP>(p, u, r, best);
-                }
 #undef FLE_FIX_BODY
-                if constexpr (!kRegAcc) release_acc();
-                if (threadIdx.x == 128 && have) p.counters[tsk] = 0u;
-                __syncwarp();
-                if (!have) ok = false;
+                    epi_finish<SWAP>(p, u, r, best);
+                    if (threadIdx.x == 128) *counter = 0u;
+                    __syncwarp();
+                }
+                if constexpr (!kRegAcc) {
+                    if (own) release_acc();
+                }
             }
 #undef FLE_LOAD_ACC
         }

@@ -368,94 +368,33 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 }
                 epi_finish<SWAP>(p, uh, r, best);
                 if constexpr (!k3x) release_acc();
-            } else if (u.kb0 != 0) {
-                // Not the tile's finisher: park this CTA's partial (column-major:
-                // element (row, col) at col * 128 + row) and count it.
-                float* slot = p.ws + static_cast<size_t>(2 * blockIdx.x + u.slot) * kBM * BN;
-                if constexpr (k3x) {
-#pragma unroll
-                    for (int lc = 0; lc < kHalf; ++lc) {
-                        if (lc < mine) {
-                            float* d = slot + static_cast<size_t>((c_lo + lc) * 32) * kBM + r;
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) __stcg(d + j * kBM, accr[lc * 32 + j]);
-                        }
-                    }
-                } else {
-#pragma unroll 1
-                    for (int lc = 0; lc < mine; ++lc) {
-                        float v[32];
-                        tmem_ld32_wait(t_acc + (c_lo + lc) * 32, v);
-                        float* d = slot + static_cast<size_t>((c_lo + lc) * 32) * kBM + r;
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) __stcg(d + j * kBM, v[j]);
-                    }
-                    release_acc();
-                }
-                __threadfence();
-                epilogue_bar_sync();
-                if (threadIdx.x == 128) atomicAdd(p.counters + 2 * u.sk_tile + rank, 1u);
-                __syncwarp();
             } else {
-                // The tile's finisher (this pair's last unit holds k-block 0):
-                // wait for the other pairs' partials of this CTA's 128 rows,
-                // add them to the own accumulator in pair order (= k order),
-                // then run the epilogue.
+                // A unit of a tile split over pairs first .. last: the same
+                // wait-free protocol as fle_gemm_kernel, per CTA of the pair
+                // (each CTA owns 128 rows of the tile and its own counter).
                 const int64_t tsk = u.sk_tile;
-                const int first = pair;
+                const int first = sk_cta_of(tsk * p.num_kb, p.sk_iters, p.sk_grid);
                 const int last = sk_cta_of((tsk + 1) * p.num_kb - 1, p.sk_iters, p.sk_grid);
+                const unsigned others = static_cast<unsigned>(last - first);
                 unsigned* counter = p.counters + 2 * tsk + rank;
-                if (threadIdx.x == 128)
-                    *last_flag = wait_count_bounded(counter, static_cast<unsigned>(last - first), abort_flag,
-                                                    p.timeout_ns, kWhereFixup)
-                                     ? 1 : 0;
-                __syncwarp();  // named barriers are .aligned: whole warps arrive
-                epilogue_bar_sync();
-                const bool have = *last_flag != 0;
-                __threadfence();
-                float best = -INFINITY;
-                auto src_of = [&](int cc, int c) {
-                    const int sl = sk_slot_of(cc, tsk, p.sk_iters, p.sk_grid, p.num_kb);
-                    return p.ws + static_cast<size_t>(2 * (2 * cc + rank) + sl) * kBM * BN +
-                           static_cast<size_t>(c * 32) * kBM + r;
-                };
-                // contributors first+1 .. last after the own accumulator; loads
-                // of up to three contributors are in flight together
-                auto add_partials = [&](int c, float (&v)[32]) {
-                    int cc = first + 1;
-                    for (; cc + 2 <= last; cc += 3) {
-                        const float* s0 = src_of(cc, c);
-                        const float* s1 = src_of(cc + 1, c);
-                        const float* s2 = src_of(cc + 2, c);
-                        float t0[32], t1[32], t2[32];
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            t0[j] = __ldcg(s0 + j * kBM);
-                            t1[j] = __ldcg(s1 + j * kBM);
-                            t2[j] = __ldcg(s2 + j * kBM);
-                        }
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = ((v[j] + t0[j]) + t1[j]) + t2[j];
-                    }
-                    for (; cc <= last; ++cc) {
-                        const float* s0 = src_of(cc, c);
-                        float t0[32];
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) t0[j] = __ldcg(s0 + j * kBM);
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] += t0[j];
-                    }
-                };
-                if (have) {
+                if (u.kb0 == 0) {
+                    if (threadIdx.x == 128) *last_flag = (ld_acquire_u32(counter) == others) ? 1 : 0;
+                    __syncwarp();  // named barriers are .aligned: whole warps arrive
+                    epilogue_bar_sync();
+                }
+                const bool own = (u.kb0 == 0) && *last_flag != 0;
+                bool fix = own;
+                if (!own) {
+                    // park this CTA's partial (column-major: element (row, col)
+                    // at col * 128 + row) and count it
+                    float* slot = p.ws + static_cast<size_t>(2 * blockIdx.x + u.slot) * kBM * BN;
                     if constexpr (k3x) {
 #pragma unroll
                         for (int lc = 0; lc < kHalf; ++lc) {
                             if (lc < mine) {
-                                float v[32];
+                                float* d = slot + static_cast<size_t>((c_lo + lc) * 32) * kBM + r;
 #pragma unroll
-                                for (int j = 0; j < 32; ++j) v[j] = accr[lc * 32 + j];
-                                add_partials(c_lo + lc, v);
-                                epi_chunk<SWAP, BN>(p, uh, r, c_lo + lc, v, best, eo);
+                                for (int j = 0; j < 32; ++j) __stcg(d + j * kBM, accr[lc * 32 + j]);
                             }
                         }
                     } else {
@@ -463,16 +402,87 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                         for (int lc = 0; lc < mine; ++lc) {
                             float v[32];
                             tmem_ld32_wait(t_acc + (c_lo + lc) * 32, v);
-                            add_partials(c_lo + lc, v);
+                            float* d = slot + static_cast<size_t>((c_lo + lc) * 32) * kBM + r;
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) __stcg(d + j * kBM, v[j]);
+                        }
+                        release_acc();
+                    }
+                    __threadfence();
+                    epilogue_bar_sync();
+                    if (threadIdx.x == 128) *last_flag = (atomicAdd(counter, 1u) == others) ? 1 : 0;
+                    __syncwarp();
+                    epilogue_bar_sync();
+                    fix = *last_flag != 0;
+                }
+                if (fix) {
+                    __threadfence();
+                    float best = -INFINITY;
+                    auto src_of = [&](int cc, int c) {
+                        const int sl = sk_slot_of(cc, tsk, p.sk_iters, p.sk_grid, p.num_kb);
+                        return p.ws + static_cast<size_t>(2 * (2 * cc + rank) + sl) * kBM * BN +
+                               static_cast<size_t>(c * 32) * kBM + r;
+                    };
+                    // contributors from..last added in order; loads of up to
+                    // three contributors are in flight together
+                    auto add_partials = [&](int c, int from, float (&v)[32]) {
+                        int cc = from;
+                        for (; cc + 2 <= last; cc += 3) {
+                            const float* s0 = src_of(cc, c);
+                            const float* s1 = src_of(cc + 1, c);
+                            const float* s2 = src_of(cc + 2, c);
+                            float t0[32], t1[32], t2[32];
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) {
+                                t0[j] = __ldcg(s0 + j * kBM);
+                                t1[j] = __ldcg(s1 + j * kBM);
+                                t2[j] = __ldcg(s2 + j * kBM);
+                            }
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] = ((v[j] + t0[j]) + t1[j]) + t2[j];
+                        }
+                        for (; cc <= last; ++cc) {
+                            const float* s0 = src_of(cc, c);
+                            float t0[32];
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) t0[j] = __ldcg(s0 + j * kBM);
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] += t0[j];
+                        }
+                    };
+                    const int from = own ? first + 1 : first;
+                    if constexpr (k3x) {
+#pragma unroll
+                        for (int lc = 0; lc < kHalf; ++lc) {
+                            if (lc < mine) {
+                                float v[32];
+#pragma unroll
+                                for (int j = 0; j < 32; ++j) v[j] = own ? accr[lc * 32 + j] : 0.0f;
+                                add_partials(c_lo + lc, from, v);
+                                epi_chunk<SWAP, BN>(p, uh, r, c_lo + lc, v, best, eo);
+                            }
+                        }
+                    } else {
+#pragma unroll 1
+                        for (int lc = 0; lc < mine; ++lc) {
+                            float v[32];
+                            if (own) {
+                                tmem_ld32_wait(t_acc + (c_lo + lc) * 32, v);
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+                            }
+                            add_partials(c_lo + lc, from, v);
                             epi_chunk<SWAP, BN>(p, uh, r, c_lo + lc, v, best, eo);
                         }
                     }
                     epi_finish<SWAP>(p, uh, r, best);
+                    if (threadIdx.x == 128) *counter = 0u;
+                    __syncwarp();
                 }
-                if constexpr (!k3x) release_acc();
-                if (threadIdx.x == 128 && have) *counter = 0u;
-                __syncwarp();
-                if (!have) ok = false;
+                if constexpr (!k3x) {
+                    if (own) release_acc();
+                }
             }
         }
     }
