@@ -254,7 +254,8 @@ int fle_test_bounded_wait(uint32_t timeout_us, void* stream);
 /*
  * Test hook for the epilogue's scalar math: out[i] = f(in[i]) for device
  * arrays of n floats, with f = erf (which = 0), exact-form GELU (1),
- * x * sigmoid(x) (2) or tanh-form GELU (3), evaluated either as the fused
+ * x * sigmoid(x) (2), tanh-form GELU (3) or exact-form GELU on |x| <= 2 by
+ * the polynomial epilogue (a) uses there (4), evaluated either as the fused
  * epilogue evaluates it (reference = 0) or with CUDA's erff/expf/tanhf and
  * IEEE division (reference = 1), so tests can bound the difference.
  * Stream-ordered.

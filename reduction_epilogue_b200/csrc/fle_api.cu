@@ -196,6 +196,15 @@ int kps_override() {
     return v;
 }
 
+// FLE_GELU_POLY=0 keeps the rational erf for epilogue (a) (comparisons).
+bool poly_disabled() {
+    static bool off = [] {
+        const char* e = std::getenv("FLE_GELU_POLY");
+        return e && e[0] == '0';
+    }();
+    return off;
+}
+
 bool pair_disabled() {
     static bool off = [] {
         const char* e = std::getenv("FLE_PAIR");
@@ -524,6 +533,10 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
     p.clamp_hi = d->clamp_hi;
     p.gelu_tanh = (d->flags & FLE_FLAG_GELU_TANH) ? 1 : 0;
     p.fold_scale = (d->flags & FLE_FLAG_FOLD_SCALE) ? 1 : 0;
+    // (a) with its GELU input clamped into [-2, 2]: the polynomial GELU
+    p.gelu_poly = (d->kind == FLE_EPI_SCALE_HARDTANH_GELU && !p.gelu_tanh && d->clamp_lo >= -2.0f &&
+                   d->clamp_hi <= 2.0f && !poly_disabled())
+                      ? 1 : 0;
     p.pool_k = pool ? d->pool_k : 1;
     p.pool_limit = pool ? (N / d->pool_k) * d->pool_k : N;
     p.vec_out = ((reinterpret_cast<uintptr_t>(out) & 15u) == 0 && N % 4 == 0) ? 1 : 0;
@@ -723,7 +736,7 @@ int fle_device_status(void* stream) {
 int fle_test_epilogue_math(const float* in, float* out, int64_t n, int32_t which, int32_t reference,
                            void* stream) {
     if (!in || !out) return FLE_ERR_NULL;
-    if (n < 0 || which < 0 || which > 3) return FLE_ERR_SHAPE;
+    if (n < 0 || which < 0 || which > 4) return FLE_ERR_SHAPE;
     DeviceInfo di;
     int st = device_info(&di);
     if (st != FLE_OK) return st;

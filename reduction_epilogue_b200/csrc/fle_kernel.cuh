@@ -69,6 +69,7 @@ struct KParams {
     int kind;
     float scale, clamp_lo, clamp_hi;
     int gelu_tanh;          // GELU in its tanh form, (a) and (c)
+    int gelu_poly;          // (a), erf form, clamp within [-2, 2]: polynomial GELU
     int fold_scale;         // (a): scale * acc + scale * b in one FMA
     int pool_k;
     int64_t pool_limit;     // columns covered by complete pool windows
@@ -210,6 +211,21 @@ __device__ __forceinline__ float gelu_tanh_form(float t) {
     return 0.5f * t * (1.0f + th);
 }
 
+// Exact-form GELU on |t| <= 2 (epilogue (a) with the pages' Hardtanh bounds):
+// t/2 + t^2 Q(t^2), Q a degree-7 least-squares fit of (t/2) erf(t/sqrt 2) / t^2
+// (gen_gelu_poly.py beside this file writes the table); eight FMAs and no
+// exponential or division.  |error| <= 1e-8 before fp32 rounding.
+__device__ __forceinline__ float gelu_poly2(float t) {
+    // Q(z), z = t^2, lowest degree first (gen_gelu_poly.py: T = 2, D = 7; fp64 max |error| 2.0e-09)
+    constexpr float kGeluPolyQ[8] = {3.989422365e-01f, -6.649000114e-02f, 9.972453726e-03f, -1.185778469e-03f,
+                                     1.142239958e-04f, -8.885020448e-06f, 5.106075654e-07f, -1.594644622e-08f};
+    const float z = t * t;
+    float q = kGeluPolyQ[7];
+#pragma unroll
+    for (int k = 6; k >= 0; --k) q = fmaf(q, z, kGeluPolyQ[k]);
+    return fmaf(z, q, 0.5f * t);
+}
+
 __device__ __forceinline__ float gelu_sel(float t, const KParams& p) {
     return p.gelu_tanh ? gelu_tanh_form(t) : gelu_erf(t);
 }
@@ -219,7 +235,7 @@ __device__ __forceinline__ float epi_apply(float y, const KParams& p) {
     if constexpr (KIND == kEpiHardtanhGelu) {
         float t = p.fold_scale ? y : y * p.scale;  // folded: y already holds s*acc + s*b
         t = fminf(fmaxf(t, p.clamp_lo), p.clamp_hi);
-        return gelu_sel(t, p);
+        return p.gelu_poly ? gelu_poly2(t) : gelu_sel(t, p);
     } else if constexpr (KIND == kEpiSwish) {
         // y * sigmoid(y); for y -> -inf, exp(-y) overflows to inf and the
         // quotient goes to 0 (the limit), never NaN.
@@ -917,8 +933,8 @@ __global__ void fle_pool_weights_kernel(const float* __restrict__ W, const float
 }
 
 // Test hook: the epilogue's scalar functions on n inputs (kind 0: erf,
-// 1: GELU, 2: swish with scale 1, 3: GELU in its tanh form), for checks
-// against CUDA's erff / expf / tanhf.
+// 1: GELU, 2: swish with scale 1, 3: GELU in its tanh form, 4: the
+// polynomial GELU of |t| <= 2), for checks against CUDA's erff / expf / tanhf.
 __global__ void fle_math_probe_kernel(const float* in, float* out, int64_t n, int which) {
     const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i >= n) return;
@@ -926,7 +942,8 @@ __global__ void fle_math_probe_kernel(const float* in, float* out, int64_t n, in
     if (which == 0) out[i] = erf_as7126(v);
     else if (which == 1) out[i] = gelu_erf(v);
     else if (which == 2) out[i] = __fdividef(v, 1.0f + __expf(-v));
-    else out[i] = gelu_tanh_form(v);
+    else if (which == 3) out[i] = gelu_tanh_form(v);
+    else out[i] = gelu_poly2(v);
 }
 __global__ void fle_math_reference_kernel(const float* in, float* out, int64_t n, int which) {
     const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -935,7 +952,8 @@ __global__ void fle_math_reference_kernel(const float* in, float* out, int64_t n
     if (which == 0) out[i] = erff(v);
     else if (which == 1) out[i] = v * 0.5f * (1.0f + erff(v * 0.70710678118654752440f));
     else if (which == 2) out[i] = v / (1.0f + expf(-v));
-    else out[i] = 0.5f * v * (1.0f + tanhf(0.79788456080286535588f * (v + 0.044715f * v * v * v)));
+    else if (which == 3) out[i] = 0.5f * v * (1.0f + tanhf(0.79788456080286535588f * (v + 0.044715f * v * v * v)));
+    else out[i] = v * 0.5f * (1.0f + erff(v * 0.70710678118654752440f));
 }
 
 // Test hook: one thread waits on a barrier nothing arrives on.

@@ -111,3 +111,23 @@ def test_binding_raises_with_status():
     with pytest.raises(fle.FleError) as e:
         fle.forward(16, 16, None, 16, d, M=-1, K=8, N=8, stream=0)
     assert e.value.status == 2
+
+
+def test_polynomial_gelu_table_is_the_generator_output():
+    # The coefficients in gelu_poly2() are what gen_gelu_poly.py fits (least
+    # squares on Chebyshev nodes, fp64 math.erf), and that fit is within 1e-8
+    # of the exact-form GELU on [-2, 2].
+    import importlib.util
+    import re
+    csrc = os.path.join(ROOT, "reduction_epilogue_b200", "csrc")
+    spec = importlib.util.spec_from_file_location("gen_gelu_poly", os.path.join(csrc, "gen_gelu_poly.py"))
+    gen = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(gen)
+    c = gen.fit()
+    assert gen.check(c) < 1e-8
+    src = open(os.path.join(csrc, "fle_kernel.cuh")).read()
+    body = src[src.index("constexpr float kGeluPolyQ[8] = {"):]
+    body = body[: body.index("};")]
+    table = [float(v) for v in re.findall(r"(-?\d\.\d+e[-+]\d+)f", body)]
+    assert len(table) == len(c) == 8
+    assert all(abs(a - b) <= 1e-6 * abs(b) for a, b in zip(table, c))
