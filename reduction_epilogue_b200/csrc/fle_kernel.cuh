@@ -230,12 +230,22 @@ __device__ __forceinline__ float gelu_sel(float t, const KParams& p) {
     return p.gelu_tanh ? gelu_tanh_form(t) : gelu_erf(t);
 }
 
-template <int KIND>
+// GELU forms of epilogue (a), chosen once per 32-value chunk so that each
+// chunk runs as straight-line code the scheduler can interleave.
+enum : int { kGeluErf = 0, kGeluTanh = 1, kGeluPoly = 2 };
+
+__device__ __forceinline__ int gelu_mode(const KParams& p) {
+    return p.gelu_tanh ? kGeluTanh : (p.gelu_poly ? kGeluPoly : kGeluErf);
+}
+
+template <int KIND, int GM = kGeluErf>
 __device__ __forceinline__ float epi_apply(float y, const KParams& p) {
     if constexpr (KIND == kEpiHardtanhGelu) {
         float t = p.fold_scale ? y : y * p.scale;  // folded: y already holds s*acc + s*b
         t = fminf(fmaxf(t, p.clamp_lo), p.clamp_hi);
-        return p.gelu_poly ? gelu_poly2(t) : gelu_sel(t, p);
+        if constexpr (GM == kGeluPoly) return gelu_poly2(t);
+        else if constexpr (GM == kGeluTanh) return gelu_tanh_form(t);
+        else return gelu_erf(t);
     } else if constexpr (KIND == kEpiSwish) {
         // y * sigmoid(y); for y -> -inf, exp(-y) overflows to inf and the
         // quotient goes to 0 (the limit), never NaN.
@@ -302,8 +312,25 @@ __device__ __forceinline__ void epi_store_direct(const KParams& p, const EpiOut&
         fold_bias32(p, n0, v);
     else
         add_bias32(p, n0, v);
+    if constexpr (KIND == kEpiHardtanhGelu) {
+        switch (gelu_mode(p)) {
+            case kGeluPoly:
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = epi_apply<KIND>(v[j], p);
+                for (int j = 0; j < 32; ++j) v[j] = epi_apply<KIND, kGeluPoly>(v[j], p);
+                break;
+            case kGeluTanh:
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = epi_apply<KIND, kGeluTanh>(v[j], p);
+                break;
+            default:
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = epi_apply<KIND, kGeluErf>(v[j], p);
+                break;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = epi_apply<KIND>(v[j], p);
+    }
     if (eo.tmap != nullptr) {
         // Row r of the block goes to staging row r; its eight 16-byte pieces
         // are placed at piece index (i ^ (r % 8)), the 128-byte swizzle the
@@ -363,10 +390,36 @@ __device__ __forceinline__ void epi_store_swapped(const KParams& p, int64_t n, i
     const bool n_ok = n < p.N;
     const bool fold = KIND == kEpiHardtanhGelu && p.fold_scale;
     const float sbn = p.scale * bn;
+    // all 32 results first (independent chains the scheduler can interleave),
+    // then the stores: for each j the warp's lanes write one 128-byte line
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-        const float o = epi_apply<KIND>(fold ? fmaf(p.scale, v[j], sbn) : v[j] + bn, p);
-        if (n_ok && m0 + j < p.M) p.out[(m0 + j) * p.N + n] = o;
+    for (int j = 0; j < 32; ++j) v[j] = fold ? fmaf(p.scale, v[j], sbn) : v[j] + bn;
+    if constexpr (KIND == kEpiHardtanhGelu) {
+        switch (gelu_mode(p)) {
+            case kGeluPoly:
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = epi_apply<KIND, kGeluPoly>(v[j], p);
+                break;
+            case kGeluTanh:
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = epi_apply<KIND, kGeluTanh>(v[j], p);
+                break;
+            default:
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = epi_apply<KIND, kGeluErf>(v[j], p);
+                break;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = epi_apply<KIND>(v[j], p);
+    }
+    if (n_ok) {
+        const int64_t ld = p.N;
+        float* o = p.out + m0 * ld + n;
+        const int64_t rows = p.M - m0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (j < rows) o[j * ld] = v[j];
     }
 }
 
@@ -883,7 +936,11 @@ __global__ void fle_bias_only_kernel(const KParams p) {
     const float y = p.bias ? p.bias[i % p.N] : 0.0f;
     float o;
     switch (p.kind) {
-        case kEpiHardtanhGelu: o = epi_apply<kEpiHardtanhGelu>(p.fold_scale ? p.scale * y : y, p); break;
+        case kEpiHardtanhGelu: {
+            const float yy = p.fold_scale ? p.scale * y : y;
+            o = p.gelu_tanh ? epi_apply<kEpiHardtanhGelu, kGeluTanh>(yy, p) : epi_apply<kEpiHardtanhGelu>(yy, p);
+            break;
+        }
         case kEpiSwish: o = epi_apply<kEpiSwish>(y, p); break;
         default: o = y; break;
     }
