@@ -4,16 +4,14 @@
 // tile (128 rows of operand A x BN rows of operand B) over a range of
 // k-blocks.  The schedule is hybrid: the first tiles are data-parallel (one
 // CTA per tile, the whole K), and the remaining tiles' k-blocks are divided
-// evenly over the first sk_grid CTAs (stream-K), so the SMs get equal shares
-// of k-blocks whatever the tile count.  The host picks the split (see
-// make_plan): shapes that stream each weight tile once spread the stream-K
-// part over every SM; shapes whose weight tiles are shared by several tiles
-// split only the last partial wave, into k-aligned parts, so the CTAs that
-// share a weight slab still walk K together and hit it in L2.  A tile whose k-range is
-// shared by several CTAs is finished by the last of them to arrive: each
-// writes its fp32 partial tile to the caller's workspace, and the last one sums
-// all partials in a fixed order (so results are bitwise reproducible) and
-// applies the epilogue.  Operand A is x and B is W
+// evenly over the first sk_grid CTAs (stream-K).  The host (make_plan) splits
+// only the last partial wave, into k-aligned parts, so CTAs that share a
+// weight slab still walk K together and hit it in L2.  A tile whose k-range
+// is split is finished without waits: the CTA holding its k-block 0 (which
+// normally ends last) adds the parked fp32 partials of the others to its own
+// accumulator; if it is not last, it parks its partial too and the last
+// arrival sums them all.  Partials are summed in a fixed order, so results
+// are bitwise reproducible.  Operand A is x and B is W
 // ("direct"), or, for small M, A is W and B is x ("swapped"), so the large
 // dimension sits on the 128-row side of the MMA; either way both operands are
 // K-major, as nn.Linear stores them.
