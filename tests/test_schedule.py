@@ -156,3 +156,17 @@ def test_workspace_matches_the_plan():
     assert lib.fle_plan_units(128, 32768, 32768, ctypes.byref(desc), 148, 0, None, 0,
                               ctypes.byref(n), ctypes.byref(g)) == 0
     assert g.value == 74  # CTA pairs, whole tiles: no workspace
+
+
+def test_uneven_last_wave_spreads_only_in_3xtf32():
+    # 1024 x 8192 x 8192 on 74 pairs: 128 tiles = 74 + 54.  The 54 tiles of
+    # the last wave cannot be split evenly (74 // 54 = 1): TF32 runs two whole
+    # waves (CTAs sharing a weight slab keep reading it together from L2),
+    # 3xTF32 spreads the last wave's k-blocks over all 74 pairs.
+    tf = fle.desc_for("avgpool_gelu_scale_rowmax", "tf32")
+    grid, per = collect(1024, 8192, 8192, tf, 148)
+    assert grid == 74 and all(int(r[5]) == 0 for rows in per for r in rows)
+    x3 = fle.desc_for("avgpool_gelu_scale_rowmax", "3xtf32")
+    grid, per = collect(1024, 8192, 8192, x3, 148)
+    load = [sum(int(r[4]) - int(r[3]) for r in rows) for rows in per]
+    assert grid == 74 and sum(load) == 128 * 256 and max(load) - min(load) <= 1
