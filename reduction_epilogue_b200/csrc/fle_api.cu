@@ -296,7 +296,8 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
             // its k-blocks over all CTAs instead: three tensor passes per byte
             // make the lost L2 reuse cheap there (1024x8192x8192 measured 10%
             // faster), while in TF32 it costs more than the idle CTAs.
-            const bool spread = hybrid || (pl.prec == fle::kPrec3xTF32 && S < 2 && pl.pair);
+            // (Only for fewer than two waves, where the idle share is large.)
+            const bool spread = hybrid || (pl.prec == fle::kPrec3xTF32 && S < 2 && pl.pair && T < 2 * G);
             if (spread && T > G) {
                 pl.dp_tiles = static_cast<int>(T - R);
                 pl.grid = static_cast<int>(G);
