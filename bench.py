@@ -87,9 +87,10 @@ def profiled_traffic(workload: str, precision: str):
     fields = {}
     with open(p) as f:
         for line in f:
-            if ":" in line and line.strip().startswith(("traffic_bytes_per_launch", "source_hash")):
-                k, v = line.split(":", 1)
-                fields[k.strip("- *`").strip()] = v.strip().strip("`")
+            item = line.strip().lstrip("-* ").strip()
+            if ":" in item and item.startswith(("traffic_bytes_per_launch", "source_hash")):
+                k, v = item.split(":", 1)
+                fields[k.strip("*` ")] = v.strip().strip("`")
     if fields.get("source_hash") != source_hash():
         return None
     try:
@@ -293,7 +294,11 @@ def run_fle(args, name, dist_ctx):
 
         def step():
             fle.forward(x, W, b, out, desc, workspace=ws, workspace_bytes=ws_bytes, stream=stream)
-    launches_per_step = (2 if problem == "avgpool_gelu_scale_rowmax" else 1) + (1 if variant == "poolfold" else 0)
+    # our kernels per call: the GEMM, a prep kernel when the plan splits K or
+    # the kind is (c), and the weight pooling of the per-call pool-fold
+    plan_sk = "sk_tiles=0 " not in fle.plan_string(*plan_shape)
+    launches_per_step = (1 + (1 if (problem == "avgpool_gelu_scale_rowmax" or plan_sk) else 0)
+                         + (1 if variant == "poolfold" else 0))
 
     input_bytes = 4 * (M * K + N * K + N)
     if variant == "poolfold_cached":
