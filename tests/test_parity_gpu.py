@@ -423,3 +423,30 @@ def test_fold_scale_option(fle, M, K, N, precision):
             atol, rtol = TOL[precision]
             err = np.abs(out.cpu().numpy().astype(np.float64) - ref)
             assert (err <= 50 * (atol + rtol * np.abs(ref))).all()
+
+
+def test_concurrent_calls_on_two_streams(fle):
+    # Two calls in flight at once on two streams, each with its own
+    # workspace (split-K plans): no CTA waits for another CTA, so the grids
+    # may share the GPU in any proportion; both results match the oracle.
+    shapes = [(16, 8192, 4096, "scale_hardtanh_gelu"), (300, 4096, 1100, "avgpool_gelu_scale_rowmax")]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    runs = []
+    for (M, K, N, problem), s in zip(shapes, streams):
+        x, W, b = synth.linear_inputs(M, K, N, seed=M + N, device="cuda")
+        d = fle.desc_for(problem, "tf32")
+        out = torch.empty((M,) if problem.startswith("avgpool") else (M, N), device="cuda")
+        wsb = fle.workspace_size(M, K, N, d)
+        assert wsb > 0  # both plans split K
+        ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+        runs.append((x, W, b, problem, out, d, ws, wsb, s))
+    torch.cuda.synchronize()
+    for _ in range(3):
+        for x, W, b, problem, out, d, ws, wsb, s in runs:
+            fle.forward(x, W, b, out, d, workspace=ws, workspace_bytes=wsb, stream=s)
+    torch.cuda.synchronize()
+    assert fle.device_status() == 0
+    for x, W, b, problem, out, d, ws, wsb, s in runs:
+        rows = synth.sample_rows(x.shape[0], 16, seed=5)
+        _assert_close(out.cpu().numpy()[rows], _oracle(x, W, b, problem, rows=rows), "tf32",
+                      f"concurrent {problem}")

@@ -12,6 +12,7 @@ import math
 from collections import defaultdict
 
 import pytest
+from hypothesis import given, settings, strategies as st
 
 import reduction_epilogue_b200 as fle
 from reduction_epilogue_b200 import build as fle_build
@@ -49,12 +50,28 @@ def collect(M, K, N, desc, sms):
 @pytest.mark.parametrize("precision", ["tf32", "3xtf32"])
 @pytest.mark.parametrize("M,K,N,problem", WORKLOADS)
 def test_schedule_covers_every_kblock_once(M, K, N, problem, precision, sms):
+    check_schedule(M, K, N, problem, precision, sms)
+
+
+@settings(max_examples=200, deadline=None, derandomize=True)
+@given(M=st.integers(1, 6000), K4=st.integers(1, 4000), N=st.integers(1, 50000),
+       problem=st.sampled_from(["scale_hardtanh_gelu", "swish_scale", "avgpool_gelu_scale_rowmax", "none"]),
+       precision=st.sampled_from(["tf32", "3xtf32"]), sms=st.sampled_from([148, 132, 16, 7]))
+def test_schedule_random_shapes(M, K4, N, problem, precision, sms):
+    # the same invariants on shapes drawn at random (K a multiple of 4, as
+    # the ABI requires)
+    if problem == "avgpool_gelu_scale_rowmax":
+        N = max(N, 16)
+    check_schedule(M, 4 * K4, N, problem, precision, sms)
+
+
+def check_schedule(M, K, N, problem, precision, sms):
     desc = fle.desc_for(problem, precision)
     grid, per_cta = collect(M, K, N, desc, sms)
     assert 1 <= grid <= sms
-    # k-blocks are 32 wide, or 16 wide for 3xTF32 on CTA pairs
+    # k-blocks are 32 wide
     num_kb = max(int(r[4]) for rows in per_cta for r in rows)
-    assert num_kb == math.ceil(K / 32) or (precision == "3xtf32" and num_kb == math.ceil(K / 16))
+    assert num_kb == math.ceil(K / 32)
     cover = defaultdict(list)  # tile -> [(kb0, kb1, cta, row)]
     for c, rows in enumerate(per_cta):
         partial_slots = []
