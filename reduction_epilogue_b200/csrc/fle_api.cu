@@ -162,16 +162,16 @@ struct Plan {
 };
 
 // Ring depth of the single-CTA kernel (mirrors Cfg::kStages).
-int stages_for(int bn, int prec, int kps, bool swap) {
+int stages_for(int bn, int prec, int kps) {
     const int stage = kps * (fle::kBM + bn) * fle::kBK * 4 * (prec == fle::kPrec3xTF32 ? 2 : 1);
-    const int s = (fle::kSmemStageBudget - (swap ? 0 : fle::kEpiWarps * fle::kEpiTileBytes)) / stage;
+    const int s = (fle::kSmemStageBudget - fle::kEpiWarps * fle::kEpiTileBytes) / stage;
     return s > 8 ? 8 : s;
 }
 
 // Ring depth of the pair kernel (mirrors PairCfg::kStages).
-int pair_stages_for(int bn, int prec, int kps, bool swap) {
+int pair_stages_for(int bn, int prec, int kps) {
     const int stage = kps * (fle::kBM + bn / 2) * fle::kBK * 4 * (prec == fle::kPrec3xTF32 ? 2 : 1);
-    const int s = (fle::kSmemStageBudget - (swap ? 0 : fle::kEpiWarps * fle::kEpiTileBytes)) / stage;
+    const int s = (fle::kSmemStageBudget - fle::kEpiWarps * fle::kEpiTileBytes) / stage;
     return s > 12 ? 12 : s;
 }
 
@@ -252,7 +252,7 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
         if (pl.swap || (pl.pair && tiles >= 2 * static_cast<int64_t>(pairs))) pl.kps = 2;
         if (kps_override() != 0) pl.kps = kps_override();
     }
-    pl.stages = pl.pair ? pair_stages_for(pl.bn, pl.prec, pl.kps, pl.swap) : stages_for(pl.bn, pl.prec, pl.kps, pl.swap);
+    pl.stages = pl.pair ? pair_stages_for(pl.bn, pl.prec, pl.kps) : stages_for(pl.bn, pl.prec, pl.kps);
 
     // The schedule runs over CTAs, or over CTA pairs in pair mode.
     const int64_t T = pl.tiles;
@@ -583,9 +583,9 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
 
     CUtensorMap ta, tb, to;
     std::memset(&to, 0, sizeof to);
-    // Direct-layout elementwise kinds store through TMA when the output rows
-    // are 16-byte multiples and the base is 16-byte aligned.
-    p.tma_out = (!pl.swap && !pool && N % 4 == 0 && (reinterpret_cast<uintptr_t>(out) & 15u) == 0) ? 1 : 0;
+    // Elementwise kinds (direct or swapped layout) store through TMA when the
+    // output rows are 16-byte multiples and the base is 16-byte aligned.
+    p.tma_out = (!pool && N % 4 == 0 && (reinterpret_cast<uintptr_t>(out) & 15u) == 0) ? 1 : 0;
     if (p.tma_out) {
         st = encode_output(&to, out, M, N);
         if (st != FLE_OK) return st;

@@ -158,7 +158,7 @@ struct Cfg {
     static constexpr int kLoadBytes = KPS * kKbBytes;                // TMA bytes per full stage
     static constexpr int kStageBytes = kLoadBytes * (PREC == kPrec3xTF32 ? 2 : 1);
     // direct layout: one 32 x 32 fp32 staging tile per epilogue warp for TMA stores
-    static constexpr int kEpiStageBytes = SWAP ? 0 : kEpiWarps * kEpiTileBytes;
+    static constexpr int kEpiStageBytes = kEpiWarps * kEpiTileBytes;
     static constexpr int kStagesRaw = (kSmemStageBudget - kEpiStageBytes) / kStageBytes;
     static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
     static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
@@ -383,7 +383,8 @@ __device__ __forceinline__ void epi_pool_direct(const KParams& p, int64_t n0, fl
 
 // Swapped layout: this thread holds output column n, rows m0..m0+31.
 template <int KIND>
-__device__ __forceinline__ void epi_store_swapped(const KParams& p, int64_t n, int64_t m0, float (&v)[32]) {
+__device__ __forceinline__ void epi_store_swapped(const KParams& p, const EpiOut& eo, int64_t n, int64_t m0,
+                                                  float (&v)[32]) {
     const float bn = (p.bias != nullptr && n < p.N) ? __ldg(p.bias + n) : 0.0f;
     const bool n_ok = n < p.N;
     const bool fold = KIND == kEpiHardtanhGelu && p.fold_scale;
@@ -410,6 +411,26 @@ __device__ __forceinline__ void epi_store_swapped(const KParams& p, int64_t n, i
     } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = epi_apply<KIND>(v[j], p);
+    }
+    if (eo.tmap != nullptr) {
+        // The warp's 32 x 32 block of out (rows m0 + j, columns n - lane +
+        // 0..31) through its staging tile and one TMA tile store: value j of
+        // this lane goes to staging row j, column lane, in the 128-byte
+        // swizzle of the tensor map (16-byte piece (lane / 4) ^ (j % 8)), so
+        // each row's 32 writes hit 32 distinct banks.  The store clips rows
+        // past M and columns past N.
+        const int lane = threadIdx.x & 31;
+        if (lane == 0) bulk_wait_read_all();  // the previous block has left this tile
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) eo.stage[j * 32 + (((lane >> 2) ^ (j & 7)) << 2) + (lane & 3)] = v[j];
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(eo.tmap, eo.stage_u32, static_cast<int32_t>(n - lane), static_cast<int32_t>(m0));
+            bulk_commit_group();
+        }
+        return;
     }
     if (n_ok) {
         const int64_t ld = p.N;
@@ -440,9 +461,9 @@ __device__ __forceinline__ void epi_chunk(const KParams& p, const Unit& u, int r
         const int64_t n = static_cast<int64_t>(u.ta) * kBM + r;
         const int64_t m0 = static_cast<int64_t>(u.tb) * BN + c * 32;
         switch (p.kind) {
-            case kEpiHardtanhGelu: epi_store_swapped<kEpiHardtanhGelu>(p, n, m0, v); break;
-            case kEpiSwish: epi_store_swapped<kEpiSwish>(p, n, m0, v); break;
-            default: epi_store_swapped<kEpiNone>(p, n, m0, v); break;
+            case kEpiHardtanhGelu: epi_store_swapped<kEpiHardtanhGelu>(p, eo, n, m0, v); break;
+            case kEpiSwish: epi_store_swapped<kEpiSwish>(p, eo, n, m0, v); break;
+            default: epi_store_swapped<kEpiNone>(p, eo, n, m0, v); break;
         }
     }
     // Stores above may branch per lane (TMA issue, bounds); the warp must be
@@ -688,8 +709,8 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         const int half = (warp - 4) >> 2;
         const int r = q * 32 + lane;  // tile row = TMEM lane of this thread
         EpiOut eo;
-        eo.tmap = (!SWAP && p.tma_out) ? &tmOut : nullptr;
-        eo.stage = reinterpret_cast<float*>(epi_stage + (SWAP ? 0 : (warp - 4) * kEpiTileBytes));
+        eo.tmap = p.tma_out ? &tmOut : nullptr;
+        eo.stage = reinterpret_cast<float*>(epi_stage + (warp - 4) * kEpiTileBytes);
         eo.stage_u32 = smem_u32(eo.stage);
         eo.row0 = 0;
         constexpr int kChunks = BN / 32;

@@ -41,8 +41,8 @@ struct PairCfg {
     static constexpr int kKbBytes = kABytes + kBBytes;
     static constexpr int kLoadBytes = KPS * kKbBytes;         // TMA bytes per full stage and CTA
     static constexpr int kStageBytes = kLoadBytes * (PREC == kPrec3xTF32 ? 2 : 1);
-    // direct layout: TMA-store staging, one 32 x 32 tile per epilogue warp
-    static constexpr int kEpiStageBytes = SWAP ? 0 : kEpiWarps * kEpiTileBytes;
+    // TMA-store staging, one 32 x 32 tile per epilogue warp
+    static constexpr int kEpiStageBytes = kEpiWarps * kEpiTileBytes;
     static constexpr int kStagesRaw = (kSmemStageBudget - kEpiStageBytes) / kStageBytes;
     static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
     static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
@@ -282,8 +282,8 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         constexpr int kHalf = (kChunks + 1) / 2;  // chunks per half
         const int c_lo = half * kHalf;
         EpiOut eo;
-        eo.tmap = (!SWAP && p.tma_out) ? &tmOut : nullptr;
-        eo.stage = reinterpret_cast<float*>(epi_stage + (SWAP ? 0 : (warp - 4) * kEpiTileBytes));
+        eo.tmap = p.tma_out ? &tmOut : nullptr;
+        eo.stage = reinterpret_cast<float*>(epi_stage + (warp - 4) * kEpiTileBytes);
         eo.stage_u32 = smem_u32(eo.stage);
         int buf = 0;
         uint32_t acc_phase = 0;
