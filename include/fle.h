@@ -93,7 +93,8 @@ typedef struct {
 enum {
     FLE_OK = 0,
     FLE_ERR_NULL = 1,        /* a required pointer is NULL                   */
-    FLE_ERR_SHAPE = 2,       /* negative size, size >= 2^31, or (c) N < pool_k */
+    FLE_ERR_SHAPE = 2,       /* negative size, size >= 2^31, M*N >= 2^40, or
+                                (c) N < pool_k                               */
     FLE_ERR_ALIGN = 3,       /* x or W not 16-byte aligned, K % 4 != 0, or
                                 out / b not 4-byte aligned                   */
     FLE_ERR_DESC = 4,        /* unknown kind/precision/flag, non-finite scale

@@ -137,6 +137,9 @@ int check_desc(const fle_epilogue_desc* d) {
 int check_shape(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d) {
     const int64_t lim = (int64_t(1) << 31);
     if (M < 0 || K < 0 || N < 0 || M >= lim || K >= lim || N >= lim) return FLE_ERR_SHAPE;
+    // 2^40 outputs (4 TiB of fp32) is far beyond any device; below it every
+    // tile count of every plan fits an int
+    if (M * N >= (int64_t(1) << 40)) return FLE_ERR_SHAPE;
     if (d->kind == FLE_EPI_AVGPOOL_GELU_SCALE_ROWMAX && N < d->pool_k) return FLE_ERR_SHAPE;
     if (K % 4 != 0) return FLE_ERR_ALIGN;
     return FLE_OK;

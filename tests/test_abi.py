@@ -96,6 +96,12 @@ def test_shape_and_alignment_errors(lib):
     assert _call(lib, 4, 8, 8, d, x=None) == 1
 
 
+def test_absurd_output_sizes_are_rejected(lib):
+    # M * N >= 2^40 outputs is rejected before anything else happens
+    d = fle.desc_for("scale_hardtanh_gelu")
+    assert _call(lib, 1 << 20, 8, 1 << 20, d) == 2  # FLE_ERR_SHAPE
+
+
 def test_empty_sizes_enqueue_nothing(lib):
     d = fle.desc_for("scale_hardtanh_gelu")
     # M == 0, or N == 0 for an elementwise kind, is valid and returns before
