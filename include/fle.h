@@ -75,7 +75,7 @@ enum {
 /* Parameters of the epilogue.  Fields that a kind does not use are ignored.
  *   scale              (a), (b), (c): multiplier
  *   clamp_lo, clamp_hi (a): Hardtanh bounds, clamp_lo <= clamp_hi
- *   pool_k, pool_stride(c): window and stride; this build supports
+ *   pool_k, pool_stride(c): window and stride; the library supports
  *                       pool_stride == pool_k with pool_k in {1,2,4,8,16,32}
  *   flags              FLE_FLAG_* options; unknown bits are FLE_ERR_DESC */
 typedef struct {
@@ -103,7 +103,7 @@ enum {
     FLE_ERR_ARCH = 6,        /* current device is not sm_100 (B200)          */
     FLE_ERR_CUDA = 7,        /* a CUDA runtime/driver call failed            */
     FLE_ERR_TIMEOUT = 8,     /* a device-side bounded wait expired           */
-    FLE_ERR_UNSUPPORTED = 9  /* valid arguments this build does not handle  */
+    FLE_ERR_UNSUPPORTED = 9  /* valid arguments the library does not handle */
 };
 
 /*

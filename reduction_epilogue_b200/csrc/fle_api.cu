@@ -491,7 +491,7 @@ const char* fle_status_string(int s) {
         case FLE_ERR_ARCH: return "device is not sm_100 (B200)";
         case FLE_ERR_CUDA: return "a CUDA call failed";
         case FLE_ERR_TIMEOUT: return "a device-side bounded wait expired";
-        case FLE_ERR_UNSUPPORTED: return "arguments valid but not supported by this build";
+        case FLE_ERR_UNSUPPORTED: return "arguments valid but not supported by the library";
         default: return "unknown status";
     }
 }
