@@ -67,3 +67,15 @@ def test_reference_arm_nonzero_rank_exits_quietly():
                         "--warmup", "3"], env=env, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0
     assert r.stdout.strip() == ""
+
+
+def test_quantile_interpolates_between_order_statistics():
+    sys.path.insert(0, ROOT)
+    import bench
+    v = [5.0, 1.0, 4.0, 2.0, 3.0]
+    assert bench.quantile(v, 0.0) == 1.0
+    assert bench.quantile(v, 1.0) == 5.0
+    assert bench.quantile(v, 0.5) == 3.0
+    assert abs(bench.quantile(v, 0.1) - 1.4) < 1e-12
+    assert abs(bench.quantile(v, 0.9) - 4.6) < 1e-12
+    assert bench.quantile([7.0], 0.9) == 7.0
