@@ -16,7 +16,6 @@ sample of rows of the same workload per step).
 from __future__ import annotations
 
 import argparse
-import hashlib
 import json
 import math
 import os
@@ -69,13 +68,10 @@ def load_peaks():
 
 
 def source_hash() -> str:
-    h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "reduction_epilogue_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, fn), "rb") as f:
-                h.update(f.read())
-    return h.hexdigest()[:12]
+    """The first 12 hex digits of the library's source hash (the sources and
+    build flags libfle.so is compiled from); profiles record it."""
+    from reduction_epilogue_b200 import build as fle_build
+    return fle_build.source_hash()[:12]
 
 
 def profiled_traffic(workload: str, precision: str):
@@ -265,17 +261,55 @@ def run_reference(args, name):
 # ----------------------------------------------------------------------------
 # the CUDA path
 # ----------------------------------------------------------------------------
-def run_fle(args, name, dist_ctx):
+def roofline(flops, nbytes, step_ms, precision, name):
+    """Roofline of the one kernel a step launches (plus its prep kernel):
+    achieved work per launch over the mean CUDA-event time per call, against
+    the measured peak of whichever bound is slower."""
+    peaks, peak_src = load_peaks()
+    tf32_peak = peaks["bf16_tflops"] * TF32_PER_BF16
+    avg_launch_s = statistics.mean(step_ms) * 1e-3
+    t_tc = flops / (tf32_peak * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    if t_tc >= t_hbm:
+        achieved = flops / avg_launch_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tf32_peak, "unit": "TFLOP/s",
+                "frac": achieved / tf32_peak,
+                "peak_source": f"{peak_src} bf16 {peaks['bf16_tflops']} TFLOP/s x 1.1/2.25 (TF32:BF16 nominal)"}
+    else:
+        achieved = nbytes / avg_launch_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "peak_source": f"{peak_src} copy bandwidth"}
+    if precision == "3xtf32":
+        # the tensor core executes three TF32 products per term, so the
+        # three-pass roofline is the slower of 3x the tensor time and HBM
+        t3 = max(3 * t_tc, t_hbm)
+        roof["roofline_3pass_time_us"] = t3 * 1e6
+        roof["frac_of_3pass"] = t3 / avg_launch_s
+    roof["traffic"] = profiled_traffic(name, precision)
+    roof["algorithmic_bytes"] = nbytes
+    roof["algorithmic_flops"] = flops
+    roof["roofline_time_us"] = max(t_tc, t_hbm) * 1e6
+    roof["kernel_us_median"] = statistics.median(step_ms) * 1e3
+    roof["kernel_us_p10"] = quantile(step_ms, 0.10) * 1e3
+    roof["kernel_us_p90"] = quantile(step_ms, 0.90) * 1e3
+    return roof
+
+
+def run_fle(args, name, dist_ctx, precision=None, brief=False):
+    """Times one workload.  Returns (on rank 0) the JSON line's dict, or with
+    brief=True a compact per-config record (no end-to-end, CPU or torch legs)."""
     import torch
 
     import reduction_epilogue_b200 as fle
     from reduction_epilogue_b200 import synth
 
     rank, world, dev = dist_ctx
+    precision = precision or args.precision
+    steps = min(args.steps, args.per_config_steps) if brief else args.steps
     M, K, N, problem = CONFIGS[name]
     variant = VARIANT.get(name)
     flops, nbytes, out_elems = algorithmic(M, K, N, problem, variant)
-    desc = fle.desc_for(problem, args.precision)
+    desc = fle.desc_for(problem, precision)
     x, W, b = synth.linear_inputs(M, K, N, seed=rank, device=dev)
     out = torch.empty((M,) if problem == "avgpool_gelu_scale_rowmax" else (M, N), device=dev)
     stream = torch.cuda.current_stream()
@@ -283,14 +317,14 @@ def run_fle(args, name, dist_ctx):
     if variant == "poolfold":
         ws_bytes = fle.workspace_size_pooled(M, K, N, desc)
         ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-        fdesc = fle.desc_for(problem, args.precision, pool_k=1)
+        fdesc = fle.desc_for(problem, precision, pool_k=1)
         plan_shape = (M, K, N // 16, fdesc)
 
         def step():
             fle.forward_pooled(x, W, b, out, desc, workspace=ws, workspace_bytes=ws_bytes, stream=stream)
     elif variant == "poolfold_cached":
         Wp, bp = fle.pool_weights(W, b, 16, stream=stream)
-        fdesc = fle.desc_for(problem, args.precision, pool_k=1)
+        fdesc = fle.desc_for(problem, precision, pool_k=1)
         ws_bytes = fle.workspace_size(M, K, N // 16, fdesc)
         ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
         plan_shape = (M, K, N // 16, fdesc)
@@ -323,14 +357,14 @@ def run_fle(args, name, dist_ctx):
     if fle.device_status(stream) != 0:
         raise RuntimeError("device status set during warm-up")
 
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(dev.index)
     with sampler:
-        for i in range(args.steps):
+        for i in range(steps):
             if flush:
                 scrub.fill_(1.0)
             starts[i].record(stream)
@@ -346,19 +380,38 @@ def run_fle(args, name, dist_ctx):
     # warm-cache figure (not the graded one) for workloads that are flushed:
     # the same steps with the inputs left in L2
     warm_ms = None
-    if flush:
+    if flush and not brief:
         w0 = torch.cuda.Event(enable_timing=True)
         w1 = torch.cuda.Event(enable_timing=True)
         step()
         w0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             step()
         w1.record(stream)
         torch.cuda.synchronize()
-        warm_ms = w0.elapsed_time(w1) / args.steps
+        warm_ms = w0.elapsed_time(w1) / steps
     total_ms = max_over_ranks(total_ms, world, dev)
-    ms_per_step = total_ms / args.steps
-    value = job_throughput_tflops(flops, world, args.steps, total_ms)
+    ms_per_step = total_ms / steps
+    value = job_throughput_tflops(flops, world, steps, total_ms)
+    roof = roofline(flops, nbytes, step_ms, precision, name)
+    plan = fle.plan_string(*plan_shape)
+    if brief:
+        del x, W, b, out, ws, scrub
+        torch.cuda.empty_cache()
+        if rank != 0:
+            return None
+        clocks = sampler.summary()
+        rec = {"workload": name, "precision": precision, "M": M, "K": K, "N": N, "epilogue": problem,
+               "steps": steps, "value": value, "unit": "TFLOP/s", "bound": roof["bound"], "frac": roof["frac"],
+               "achieved": roof["achieved"], "achieved_unit": roof["unit"], "peak": roof["peak"],
+               "roofline_time_us": roof["roofline_time_us"], "kernel_us_median": roof["kernel_us_median"],
+               "kernel_us_p10": roof["kernel_us_p10"], "kernel_us_p90": roof["kernel_us_p90"],
+               "traffic": roof["traffic"], "plan": plan,
+               "l2": "flushed between steps" if flush else "inputs larger than L2",
+               "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")}}
+        if "frac_of_3pass" in roof:
+            rec["frac_of_3pass"] = roof["frac_of_3pass"]
+        return rec
 
     # end to end through the public call: pinned host inputs in, result out
     e2e = None
@@ -367,7 +420,7 @@ def run_fle(args, name, dist_ctx):
         Wh = W.cpu().pin_memory()
         bh = b.cpu().pin_memory()
         outh = torch.empty(out.shape, dtype=torch.float32).pin_memory()
-        e2e_steps = max(1, min(args.steps, args.e2e_steps))
+        e2e_steps = max(1, min(steps, args.e2e_steps))
         copy_w = variant != "poolfold_cached"  # cached pooled weights stay on the device
 
         def h2d():
@@ -397,35 +450,6 @@ def run_fle(args, name, dist_ctx):
                "h2d_bytes_per_step": (4 * (M * K + N * K + N) if copy_w else 4 * M * K),
                "d2h_bytes_per_step": 4 * out_elems, "steps": e2e_steps}
 
-    # roofline of the dominant (only) kernel
-    peaks, peak_src = load_peaks()
-    tf32_peak = peaks["bf16_tflops"] * TF32_PER_BF16
-    avg_launch_s = statistics.mean(step_ms) * 1e-3
-    t_tc = flops / (tf32_peak * 1e12)
-    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
-    traffic = profiled_traffic(name, args.precision)
-    if t_tc >= t_hbm:
-        achieved = flops / avg_launch_s / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": tf32_peak, "unit": "TFLOP/s",
-                "frac": achieved / tf32_peak,
-                "peak_source": f"{peak_src} bf16 {peaks['bf16_tflops']} TFLOP/s x 1.1/2.25 (TF32:BF16 nominal)"}
-    else:
-        achieved = nbytes / avg_launch_s / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "peak_source": f"{peak_src} copy bandwidth"}
-    if args.precision == "3xtf32":
-        # the tensor core executes three TF32 products per term, so the
-        # three-pass roofline is the slower of 3x the tensor time and HBM
-        t3 = max(3 * t_tc, t_hbm)
-        roof["roofline_3pass_time_us"] = t3 * 1e6
-        roof["frac_of_3pass"] = t3 / avg_launch_s
-    roof["traffic"] = traffic
-    roof["algorithmic_bytes"] = nbytes
-    roof["algorithmic_flops"] = flops
-    roof["roofline_time_us"] = max(t_tc, t_hbm) * 1e6
-    roof["kernel_us_median"] = statistics.median(step_ms) * 1e3
-    roof["kernel_us_p10"] = quantile(step_ms, 0.10) * 1e3
-    roof["kernel_us_p90"] = quantile(step_ms, 0.90) * 1e3
     if warm_ms is not None:
         roof["kernel_us_warm_l2"] = warm_ms * 1e3
 
@@ -433,7 +457,7 @@ def run_fle(args, name, dist_ctx):
     # GPU -- torch.addmm (cuBLAS, TF32 allowed) followed by the epilogue as
     # separate eager elementwise ops.
     context = None
-    if args.context_torch and variant is None and args.precision == "tf32":
+    if args.context_torch and variant is None and precision == "tf32":
         import torch.nn.functional as F
         prev = torch.backends.cuda.matmul.allow_tf32
         torch.backends.cuda.matmul.allow_tf32 = True
@@ -454,12 +478,12 @@ def run_fle(args, name, dist_ctx):
         c0 = torch.cuda.Event(enable_timing=True)
         c1 = torch.cuda.Event(enable_timing=True)
         c0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             torch_step()
         c1.record(stream)
         torch.cuda.synchronize()
         torch.backends.cuda.matmul.allow_tf32 = prev
-        t_ms = c0.elapsed_time(c1) / args.steps
+        t_ms = c0.elapsed_time(c1) / steps
         context = {"what": "torch.addmm (cuBLAS TF32) + eager epilogue ops, same inputs and GPU",
                    "ms_per_step": t_ms, "tflops": flops / (t_ms * 1e-3) / 1e12,
                    "fused_speedup": t_ms / ms_per_step}
@@ -475,26 +499,43 @@ def run_fle(args, name, dist_ctx):
         cpu = {"value": 2.0 * R * N * K / t / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
                "kind": "oracle", "sample": f"rows 0..{R - 1} of {M} (full N={N}, K={K}); {t:.1f} s"}
 
+    line = None
     if rank == 0:
         line = {
             "impl": "fle", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "tf32" if args.precision == "tf32" else "3xtf32",
+            "steps": steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "tf32" if precision == "tf32" else "3xtf32",
             "data": "synthetic",
-            "config": {"workload": name, "M": M, "K": K, "N": N, "epilogue": problem, "precision": args.precision,
+            "config": {"workload": name, "M": M, "K": K, "N": N, "epilogue": problem, "precision": precision,
                        "l2": "flushed between steps" if flush else "inputs larger than L2",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "plan": fle.plan_string(*plan_shape),
+                       "plan": plan,
                        **({"variant": variant, "effective_tflops_of_unpooled_problem":
-                           2.0 * M * N * K * world * args.steps / (total_ms * 1e-3) / 1e12} if variant else {})},
+                           2.0 * M * N * K * world * steps / (total_ms * 1e-3) / 1e12} if variant else {})},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": sampler.summary(),
-            "gpu_launches": launches_per_step * args.steps,
+            "gpu_launches": launches_per_step * steps,
         }
         if context is not None:
             line["context_torch"] = context
-        print(json.dumps(line), flush=True)
     del x, W, b, out, ws, scrub
     torch.cuda.empty_cache()
+    return line
+
+
+# The other workloads measured in the default run, each with its own timed
+# region, after the headline: (config, precision).
+PER_CONFIG = [
+    ("linear128x1024x1024_hardtanh_gelu", "tf32"),
+    ("linear1024x8192x8192_pool16_gelu_rowmax", "tf32"),
+    ("linear128x32768x32768_swish", "tf32"),
+    ("sweep_m16_k8192_n8192_hardtanh_gelu", "tf32"),
+    ("sweep_m64_k8192_n8192_hardtanh_gelu", "tf32"),
+    ("sweep_m256_k8192_n8192_hardtanh_gelu", "tf32"),
+    ("sweep_m1024_k8192_n8192_hardtanh_gelu", "tf32"),
+    ("sweep_m4096_k8192_n8192_hardtanh_gelu", "tf32"),
+    ("linear2048x8192x8192_hardtanh_gelu", "3xtf32"),
+    ("linear128x32768x32768_swish", "3xtf32"),
+]
 
 
 def main():
@@ -502,7 +543,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(CONFIGS))
+    ap.add_argument("--config", default=None, choices=sorted(CONFIGS),
+                    help=f"one workload (default {DEFAULT_CONFIG}, followed by the per-config records)")
     ap.add_argument("--all", action="store_true", help="one line per config")
     ap.add_argument("--shape", default=None,
                     help="M,K,N,problem: a custom workload (for profiling smaller cases)")
@@ -514,10 +556,17 @@ def main():
                     help="also time torch.addmm + eager epilogue ops on the same inputs (context)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work to time")
+    ap.add_argument("--per-config-steps", type=int, default=20,
+                    help="timed steps of each per-config record (at most --steps)")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="the default run without the per-config records")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    names = sorted(CONFIGS) if args.all else [args.config]
+    # The default run (no workload named) times the headline workload and,
+    # on one GPU, adds a record of every other benchmark workload to its line.
+    per_config = args.config is None and not args.all and not args.shape and not args.no_per_config
+    names = sorted(CONFIGS) if args.all else [args.config or DEFAULT_CONFIG]
     if args.shape:
         M, K, N, problem = args.shape.split(",")
         name = f"custom_m{M}_k{K}_n{N}_{problem}"
@@ -544,7 +593,16 @@ def main():
     fle.load()
     try:
         for n in names:
-            run_fle(args, n, (rank, world, dev))
+            line = run_fle(args, n, (rank, world, dev))
+            if per_config and world == 1:
+                recs = []
+                for pn, prec in PER_CONFIG:
+                    if (pn, prec) == (n, args.precision):
+                        continue
+                    recs.append(run_fle(args, pn, (rank, world, dev), precision=prec, brief=True))
+                line["per_config"] = recs
+            if line is not None:
+                print(json.dumps(line), flush=True)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

@@ -103,7 +103,9 @@ enum {
     FLE_ERR_ARCH = 6,        /* current device is not sm_100 (B200)          */
     FLE_ERR_CUDA = 7,        /* a CUDA runtime/driver call failed            */
     FLE_ERR_TIMEOUT = 8,     /* a device-side bounded wait expired           */
-    FLE_ERR_UNSUPPORTED = 9  /* valid arguments the library does not handle */
+    FLE_ERR_UNSUPPORTED = 9, /* valid arguments the library does not handle */
+    FLE_ERR_PROTOCOL = 10    /* a barrier-protocol check failed (only the checking
+                                build, -DFLE_CHECK_BARRIERS, makes these checks) */
 };
 
 /*
@@ -242,27 +244,12 @@ int fle_forward_noalloc(const float* x, const float* W, const float* b,
 /* Library ABI version (major * 10000 + minor * 100 + patch). */
 int fle_version(void);
 
-/*
- * Test hook for the bounded-wait machinery: launches one CTA whose thread
- * waits on a shared-memory barrier that nothing ever arrives on, with a wait
- * limit of timeout_us microseconds.  The wait gives up, records
- * FLE_ERR_TIMEOUT in the device status word and the kernel returns normally,
- * so the context stays usable.  Returns the launch status; read the recorded
- * status with fle_device_status().
- */
-int fle_test_bounded_wait(uint32_t timeout_us, void* stream);
+/* The SHA-256 (hex) of the sources and build flags this library was compiled
+ * from; the Python binding refuses a library whose hash does not match the
+ * sources beside it.  Static text, never NULL. */
+const char* fle_source_hash(void);
 
-/*
- * Test hook for the epilogue's scalar math: out[i] = f(in[i]) for device
- * arrays of n floats, with f = erf (which = 0), exact-form GELU (1),
- * x * sigmoid(x) (2), tanh-form GELU (3) or exact-form GELU on |x| <= 2 by
- * the polynomial epilogue (a) uses there (4), evaluated either as the fused
- * epilogue evaluates it (reference = 0) or with CUDA's erff/expf/tanhf and
- * IEEE division (reference = 1), so tests can bound the difference.
- * Stream-ordered.
- */
-int fle_test_epilogue_math(const float* in, float* out, int64_t n, int32_t which, int32_t reference,
-                           void* stream);
+/* Test and diagnostic hooks are declared in fle_testing.h. */
 
 #ifdef __cplusplus
 }

@@ -22,7 +22,10 @@ __all__ = [
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-_LIB = os.path.join(_PKG, "lib", "libfle.so")
+# FLE_BUILD=check selects the barrier-checking build of the same sources
+# (-DFLE_CHECK_BARRIERS: protocol checks record FLE_ERR_PROTOCOL); tests only.
+_CHECK = os.environ.get("FLE_BUILD", "") == "check"
+_LIB = os.path.join(_PKG, "lib", "libfle_check.so" if _CHECK else "libfle.so")
 
 # Values mirror include/fle.h.
 EPI_SCALE_HARDTANH_GELU = 0
@@ -38,7 +41,7 @@ FLE_OK = 0
 STATUS_NAMES = {
     0: "FLE_OK", 1: "FLE_ERR_NULL", 2: "FLE_ERR_SHAPE", 3: "FLE_ERR_ALIGN", 4: "FLE_ERR_DESC",
     5: "FLE_ERR_WORKSPACE", 6: "FLE_ERR_ARCH", 7: "FLE_ERR_CUDA", 8: "FLE_ERR_TIMEOUT",
-    9: "FLE_ERR_UNSUPPORTED",
+    9: "FLE_ERR_UNSUPPORTED", 10: "FLE_ERR_PROTOCOL",
 }
 
 # The pages' three problems: epilogue kind and constants.
@@ -85,6 +88,11 @@ def load():
     if not os.path.exists(_LIB):
         raise FileNotFoundError(
             f"{_LIB} is missing; build it with `python -m reduction_epilogue_b200.build`")
+    from . import build as _build
+    if _build.sources_present() and _build.built_hash(_LIB) != _build.source_hash(_CHECK):
+        raise RuntimeError(
+            f"{_LIB} was not built from the sources beside it; rebuild it with "
+            "`python -m reduction_epilogue_b200.build`")
     lib = ctypes.CDLL(_LIB)
     i64, vp, sz = ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
     lib.fle_forward.argtypes = [vp, vp, vp, i64, i64, i64, ctypes.POINTER(EpilogueDesc), vp, vp, sz, vp]
@@ -108,8 +116,14 @@ def load():
     lib.fle_workspace_size_pooled.restype = sz
     lib.fle_forward_pooled.argtypes = [vp, vp, vp, i64, i64, i64, ctypes.POINTER(EpilogueDesc), vp, vp, sz, vp]
     lib.fle_forward_pooled.restype = ctypes.c_int
+    lib.fle_source_hash.argtypes = []
+    lib.fle_source_hash.restype = ctypes.c_char_p
     lib.fle_test_bounded_wait.argtypes = [ctypes.c_uint32, vp]
     lib.fle_test_bounded_wait.restype = ctypes.c_int
+    lib.fle_test_set_finisher.argtypes = [ctypes.c_int32]
+    lib.fle_test_set_finisher.restype = ctypes.c_int
+    lib.fle_test_finisher_counts.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32, vp]
+    lib.fle_test_finisher_counts.restype = ctypes.c_int
     _lib = lib
     return lib
 

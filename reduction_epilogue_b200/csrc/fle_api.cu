@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "fle.h"
+#include "fle_testing.h"
 #include "fle_kernel.cuh"
 #include "fle_kernel_pair.cuh"
 
@@ -209,12 +210,41 @@ bool poly_disabled() {
     return off;
 }
 
-bool pair_disabled() {
-    static bool off = [] {
-        const char* e = std::getenv("FLE_PAIR");
-        return e && e[0] == '0';
+// FLE_PAIR_BN=224 or 256 fixes the direct pair tile's width (comparisons).
+int pair_bn_override() {
+    static int v = [] {
+        const char* e = std::getenv("FLE_PAIR_BN");
+        const int n = e ? std::atoi(e) : 0;
+        return (n == fle::kPairBN || n == fle::kPairBNNarrow) ? n : 0;
     }();
-    return off;
+    return v;
+}
+
+// FLE_PAIR=0 keeps every plan on one-CTA tiles; FLE_PAIR=1 puts every
+// swapped plan on CTA pairs (comparisons).
+int pair_override() {
+    static int v = [] {
+        const char* e = std::getenv("FLE_PAIR");
+        return (e && (e[0] == '0' || e[0] == '1')) ? e[0] - '0' : -1;
+    }();
+    return v;
+}
+bool pair_disabled() { return pair_override() == 0; }
+
+// Waves of a plan of T tiles on G (pairs of) CTAs in units of one tile's
+// time, counting the last partial wave of R tiles as 1/S when make_plan
+// splits it S ways (S >= 2, k-aligned parts), as R/G when it spreads that
+// wave's k-blocks over all G (spread: the 3xTF32 rule of make_plan), else as
+// a whole wave.
+double plan_waves(int64_t T, int64_t G, int num_kb, int64_t min_iters, bool spread) {
+    const int64_t R = T % G;
+    double w = static_cast<double>(T / G);
+    if (R == 0) return w;
+    if (num_kb < 4 * min_iters) return w + 1.0;
+    const int64_t S = std::min<int64_t>(G / R, num_kb / min_iters);
+    if (S >= 2) return w + 1.0 / static_cast<double>(S);
+    if (spread && T > G && T < 2 * G) return w + static_cast<double>(R) / static_cast<double>(G);
+    return w + 1.0;
 }
 
 // sms: SMs of the device; pairs: co-resident CTA pairs of the pair kernel.
@@ -229,14 +259,39 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
     // is faster).
     const bool pairs_ok = pairs > 0 && !pair_disabled();
     if (pl.swap)
-        pl.pair = pairs_ok && pl.prec == fle::kPrecTF32 && (N + fle::kPairBM - 1) / fle::kPairBM >= pairs;
+        pl.pair = pairs_ok && ((pl.prec == fle::kPrecTF32 && (N + fle::kPairBM - 1) / fle::kPairBM >= pairs) ||
+                               pair_override() == 1);
     else
         pl.pair = pairs_ok && M > 128;
     int tile_m = pl.pair ? fle::kPairBM : fle::kBM;
+    // the stream-K minimum is 16 k-blocks of 32 (512 of K) per CTA
+    // (FLE_MIN_KB overrides it for comparisons)
+    static const int64_t min_kb_env = [] {
+        const char* e = std::getenv("FLE_MIN_KB");
+        const long v = e ? std::atol(e) : 0;
+        return static_cast<int64_t>(v > 0 ? v : 0);
+    }();
+    const int64_t min_iters = min_kb_env > 0 ? min_kb_env : kMinSkIters;
+    const int num_kb = static_cast<int>((K + fle::kBK - 1) / fle::kBK);
     if (pl.swap) {
         pl.bn = M <= 32 ? 32 : (M <= 64 ? 64 : 128);
     } else if (pl.pair) {
-        pl.bn = fle::kPairBN;
+        // 256 or 224 B rows per pair tile: the narrower tile when it fills
+        // the waves enough better (time ~ columns per tile x waves; e.g.
+        // 1024 x 8192 x 8192: 128 tiles of 256 = 2 waves on 74 pairs, 148
+        // tiles of 224 = 2 full waves, 12.5% fewer columns per pair)
+        // (in 3xTF32 a 256-wide plan that spreads its uneven last wave over
+        // all pairs measured faster than the two whole waves of 224: 805
+        // against 850 us on 1024 x 8192 x 8192)
+        const int64_t ta = (M + fle::kPairBM - 1) / fle::kPairBM;
+        const int64_t G = pairs;
+        const bool spread = pl.prec == fle::kPrec3xTF32;
+        const double c256 = fle::kPairBN *
+                            plan_waves(ta * ((N + fle::kPairBN - 1) / fle::kPairBN), G, num_kb, min_iters, spread);
+        const double c224 = fle::kPairBNNarrow *
+                            plan_waves(ta * ((N + fle::kPairBNNarrow - 1) / fle::kPairBNNarrow), G, num_kb, min_iters, spread);
+        pl.bn = (c224 < 0.97 * c256) ? fle::kPairBNNarrow : fle::kPairBN;
+        if (pair_bn_override() != 0) pl.bn = pair_bn_override();
     } else {
         pl.bn = (pl.prec == fle::kPrec3xTF32) ? 128 : 256;
     }
@@ -266,14 +321,6 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
     const bool force_dp = std::strcmp(ov, "dp") == 0;
     const bool force_sk = std::strcmp(ov, "sk") == 0;
     const bool hybrid = std::strcmp(ov, "hybrid") == 0;
-    // the stream-K minimum is 16 k-blocks of 32 (512 of K) per CTA
-    // (FLE_MIN_KB overrides it for comparisons)
-    static const int64_t min_kb_env = [] {
-        const char* e = std::getenv("FLE_MIN_KB");
-        const long v = e ? std::atol(e) : 0;
-        return static_cast<int64_t>(v > 0 ? v : 0);
-    }();
-    const int64_t min_iters = min_kb_env > 0 ? min_kb_env : kMinSkIters * fle::kBK / pl.bk;
     pl.dp_tiles = static_cast<int>(T);
     pl.grid = static_cast<int>(T < G ? T : G);
     pl.sk_grid = 0;
@@ -394,6 +441,11 @@ cudaError_t dispatch(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& t
     using namespace fle;
     const bool tf32 = pl.prec == kPrecTF32;
     const bool two = pl.kps == 2;  // TF32 only
+    if (pl.pair && !pl.swap && pl.bn == kPairBNNarrow) {
+        if (!tf32) return launch_gemm_pair<kPrec3xTF32, 1, kPairBNNarrow>(ta, tb, to, p, pl.grid, after_prep, st);
+        return two ? launch_gemm_pair<kPrecTF32, 2, kPairBNNarrow>(ta, tb, to, p, pl.grid, after_prep, st)
+                   : launch_gemm_pair<kPrecTF32, 1, kPairBNNarrow>(ta, tb, to, p, pl.grid, after_prep, st);
+    }
     if (pl.pair && !pl.swap) {
         if (!tf32) return launch_gemm_pair<kPrec3xTF32, 1>(ta, tb, to, p, pl.grid, after_prep, st);
         return two ? launch_gemm_pair<kPrecTF32, 2>(ta, tb, to, p, pl.grid, after_prep, st)
@@ -447,6 +499,9 @@ uint64_t timeout_ns() {
     return t;
 }
 
+// Finisher mode of split tiles (fle_test_set_finisher); FLE_FINISH_AUTO in use.
+std::atomic<int> g_finish_mode{FLE_FINISH_AUTO};
+
 bool log_enabled() {
     static bool on = [] {
         const char* e = std::getenv("FLE_LOG");
@@ -479,7 +534,14 @@ int plan_to_string(const Plan& pl, char* buf, size_t n) {
 
 extern "C" {
 
-int fle_version(void) { return 100; }
+int fle_version(void) { return 200; }
+
+#ifndef FLE_SOURCE_HASH
+#define FLE_SOURCE_HASH "unknown"
+#endif
+// The marker prefix lets the build script find the hash in the built file.
+static const char kSourceHashTag[] = "fle-source-sha256:" FLE_SOURCE_HASH;
+const char* fle_source_hash(void) { return kSourceHashTag + 18; }
 
 const char* fle_status_string(int s) {
     switch (s) {
@@ -493,6 +555,7 @@ const char* fle_status_string(int s) {
         case FLE_ERR_CUDA: return "a CUDA call failed";
         case FLE_ERR_TIMEOUT: return "a device-side bounded wait expired";
         case FLE_ERR_UNSUPPORTED: return "arguments valid but not supported by the library";
+        case FLE_ERR_PROTOCOL: return "a barrier-protocol check failed (checking build)";
         default: return "unknown status";
     }
 }
@@ -557,6 +620,11 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
     p.vec_out = ((reinterpret_cast<uintptr_t>(out) & 15u) == 0 && N % 4 == 0) ? 1 : 0;
     p.vec_bias = (b && (reinterpret_cast<uintptr_t>(b) & 15u) == 0) ? 1 : 0;
     p.timeout_ns = timeout_ns();
+    switch (g_finish_mode.load(std::memory_order_relaxed)) {
+        case FLE_FINISH_OWN: p.sk_finish = fle::kFinishOwn; break;
+        case FLE_FINISH_LAST: p.sk_finish = fle::kFinishPark; break;
+        default: p.sk_finish = fle::kFinishAuto; break;
+    }
 
     if (K == 0) {
         const int64_t n = pool ? M : M * N;
@@ -764,6 +832,25 @@ int fle_test_epilogue_math(const float* in, float* out, int64_t n, int32_t which
     else
         fle::fle_math_probe_kernel<<<blocks, threads, 0, s>>>(in, out, n, which);
     return cudaGetLastError() == cudaSuccess ? FLE_OK : FLE_ERR_CUDA;
+}
+
+int fle_test_set_finisher(int32_t mode) {
+    if (mode != FLE_FINISH_AUTO && mode != FLE_FINISH_OWN && mode != FLE_FINISH_LAST) return -1;
+    return g_finish_mode.exchange(mode);
+}
+
+int fle_test_finisher_counts(uint32_t* counts, int32_t reset, void* stream) {
+    if (!counts) return FLE_ERR_NULL;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FLE_ERR_CUDA;
+    unsigned h[2] = {0, 0};
+    if (cudaMemcpyFromSymbol(h, fle::g_finish_count, sizeof h) != cudaSuccess) return FLE_ERR_CUDA;
+    counts[0] = h[0];
+    counts[1] = h[1];
+    if (reset) {
+        const unsigned z[2] = {0, 0};
+        if (cudaMemcpyToSymbol(fle::g_finish_count, z, sizeof z) != cudaSuccess) return FLE_ERR_CUDA;
+    }
+    return FLE_OK;
 }
 
 int fle_test_bounded_wait(uint32_t timeout_us, void* stream) {

@@ -44,6 +44,9 @@ constexpr int kSmemStageBudget = 229376;  // bytes of shared memory for stages (
 
 enum : int { kEpiHardtanhGelu = 0, kEpiSwish = 1, kEpiPoolMax = 2, kEpiNone = 3 };
 enum : int { kPrec3xTF32 = 0, kPrecTF32 = 1 };
+// Who finishes a tile whose k-range is split over CTAs (KParams::sk_finish).
+// kFinishAuto is the product behaviour; the other two pin one branch for tests.
+enum : int { kFinishAuto = 0, kFinishOwn = 1, kFinishPark = 2 };
 
 // Wait-site identifiers recorded with a timeout.
 enum : unsigned {
@@ -71,6 +74,7 @@ struct KParams {
     int fold_scale;         // (a): scale * acc + scale * b in one FMA
     int pool_k;
     int64_t pool_limit;     // columns covered by complete pool windows
+    int sk_finish;          // kFinishAuto / kFinishOwn / kFinishPark
     int vec_out;            // out 16-byte aligned and N % 4 == 0
     int vec_bias;           // bias 16-byte aligned
     int tma_out;            // direct layout: write out through TMA tile stores
@@ -166,7 +170,7 @@ struct Cfg {
     // barriers: full, conv, empty per stage; accf, acce per buffer; drain
     static constexpr int kNumBars = 3 * kStages + 4 + 1;
     static constexpr int kSmemBytes =
-        1024 /*align slack*/ + kStages * kStageBytes + kEpiStageBytes + kNumBars * 8 + 32;
+        1024 /*align slack*/ + kStages * kStageBytes + kEpiStageBytes + kNumBars * 8 + 32 + (kCheckBarriers ? 64 : 0);
     static_assert(kStages >= 2, "need at least two stages");
     static_assert(KPS == 1 || KPS == 2, "one or two k-blocks per stage");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128 is a multiple of 16 in [16,256]");
@@ -493,6 +497,28 @@ __device__ __forceinline__ void epilogue_bar_sync() {
     asm volatile("bar.sync 1, 256;" ::: "memory");
 }
 
+// Limit of the test-only wait of kFinishOwn (after it the CTA parks as usual).
+constexpr uint64_t kFinishOwnWaitNs = 50000000ull;
+
+// Whether the CTA holding k-block 0 of a shared tile finishes it from its own
+// accumulator: only when all `others` contributors have parked their partials
+// (arrival counter == others).  kFinishPark never does; kFinishOwn first
+// waits, up to a fixed limit, for the others to arrive (a test mode: every
+// contributor of a tile is resident together in the plans this library
+// makes, so the wait ends; if it does not, the CTA parks, which is correct).
+__device__ __forceinline__ bool sk_take_own(const KParams& p, const unsigned* counter, unsigned others) {
+    if (p.sk_finish == kFinishPark) return false;
+    unsigned c = ld_acquire_u32(counter);
+    if (c != others && p.sk_finish == kFinishOwn) {
+        const uint64_t t0 = global_timer_ns();
+        while (c != others && global_timer_ns() - t0 < kFinishOwnWaitNs) {
+            __nanosleep(200);
+            c = ld_acquire_u32(counter);
+        }
+    }
+    return c == others;
+}
+
 // ----------------------------------------------------------------------------
 // The kernel
 // ----------------------------------------------------------------------------
@@ -515,7 +541,14 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     uint64_t* bars = reinterpret_cast<uint64_t*>(epi_stage + C::kEpiStageBytes);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    // two slots used in turn: a slot is written again only after every
+    // epilogue thread has passed a later barrier, so after its read
     volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+    // checking build: the work tag of each stage and accumulator buffer
+    volatile uint32_t* stage_tag = reinterpret_cast<volatile uint32_t*>(tmem_slot + 8);
+    volatile uint32_t* acc_tag = stage_tag + 12;
+    (void)stage_tag;
+    (void)acc_tag;
 
     auto bar_full = [&](int s) { return smem_u32(bars + s); };
     auto bar_conv = [&](int s) { return smem_u32(bars + S + s); };
@@ -574,6 +607,10 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         ok = false;
                         break;
                     }
+                    if constexpr (kCheckBarriers) {
+                        if (mbar_test_wait(bar_full(stage), phase)) record_error(kErrProtocol, kWhereProdEmpty);
+                        stage_tag[stage] = work_tag(u.t, kb);
+                    }
                     mbar_arrive_expect_tx(bar_full(stage), n * C::kKbBytes);
                     for (int j = 0; j < n; ++j) {
                         tma_load_2d(sA(stage) + j * C::kABytes, &tmA, bar_full(stage), (kb + j) * kBK, u.ta * kBM);
@@ -588,7 +625,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 const int s = static_cast<int>(f % S);
                 const uint32_t ph = static_cast<uint32_t>((f / S) & 1);
                 volatile int never = 0;
-                mbar_wait_bounded(bar_full(s), ph, &never, p.timeout_ns, kWhereProdDrain);
+                mbar_wait_bounded(bar_full(s), ph, &never, kDrainTimeoutNs, kWhereProdDrain);
             }
         }
     } else if (warp == 1) {
@@ -612,6 +649,10 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     break;
                 }
                 tc_fence_after_sync();
+                if constexpr (kCheckBarriers) {
+                    acc_tag[buf] = work_tag(u.t, kc);
+                    __threadfence_block();
+                }
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
                 for (int kb = kc; kb < kce; kb += KPS) {
                     const int n = (kce - kb < KPS) ? kce - kb : KPS;  // k-blocks in this stage
@@ -621,6 +662,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         break;
                     }
                     tc_fence_after_sync();
+                    if constexpr (kCheckBarriers) check_tag(stage_tag[stage], work_tag(u.t, kb), kWhereMmaFull);
                     for (int j = 0; j < n; ++j) {
                         const uint64_t a_hi = smem_desc_sw128(sA(stage) + j * C::kABytes);
                         const uint64_t b_hi = smem_desc_sw128(sB(stage) + j * C::kBBytes);
@@ -652,7 +694,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             // All issued MMAs must be complete before TMEM is released.
             mma_commit(bar_drain);
             volatile int never = 0;
-            mbar_wait_bounded(bar_drain, 0, &never, p.timeout_ns, kWhereDrain);
+            mbar_wait_bounded(bar_drain, 0, &never, kDrainTimeoutNs, kWhereDrain);
         }
         __syncwarp();
     } else if (warp < 4) {
@@ -672,6 +714,9 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         got = mbar_wait_bounded(bar_full(stage), phase, abort_flag, p.timeout_ns, kWhereConvFull);
                     got = __shfl_sync(0xffffffffu, got, 0);
                     if (!got) { ok = false; break; }
+                    if constexpr (kCheckBarriers) {
+                        if (lane == 0) check_tag(stage_tag[stage], work_tag(u.t, kb), kWhereConvFull);
+                    }
                     // hi = x with the low 13 mantissa bits cleared (a TF32
                     // value); lo = x - hi (exact in fp32) goes to the same
                     // offset in the lo half.  The tensor core reads the raw x
@@ -724,6 +769,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         // zero, whose bias would otherwise grow with the length of K.
         constexpr bool kRegAcc = (PREC == kPrec3xTF32);
         float accr[kRegAcc ? kHalf * 32 : 1];
+        int fsel = 0;  // next last_flag slot (the same in every epilogue thread)
         Sched sc;
         sc.init(p, blockIdx.x, gridDim.x);
         Unit u;
@@ -736,10 +782,14 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             const int mine = nchunks - c_lo < 0 ? 0 : (nchunks - c_lo > kHalf ? kHalf : nchunks - c_lo);
             eo.row0 = static_cast<int64_t>(u.ta) * kBM + q * 32;
 
-            auto wait_acc = [&]() -> bool {
+            auto wait_acc = [&](int kc) -> bool {
                 int got = 0;
-                if (lane == 0)
+                if (lane == 0) {
                     got = mbar_wait_bounded(bar_accf(buf), acc_phase, abort_flag, p.timeout_ns, kWhereEpiAccFull);
+                    if constexpr (kCheckBarriers) {
+                        if (got) check_tag(acc_tag[buf], work_tag(u.t, kc), kWhereEpiAccFull);
+                    }
+                }
                 got = __shfl_sync(0xffffffffu, got, 0);
                 if (got) tc_fence_after_sync();
                 return got != 0;
@@ -761,7 +811,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 #pragma unroll
                 for (int j = 0; j < (kRegAcc ? kHalf * 32 : 1); ++j) accr[j] = 0.0f;
                 for (int kc = u.kb0; kc < u.kb1; kc += kChunkKb) {
-                    if (!wait_acc()) { ok = false; break; }
+                    if (!wait_acc(kc)) { ok = false; break; }
                     const uint32_t tr = t_row();
 #pragma unroll
                     for (int lc = 0; lc < kHalf; ++lc) {
@@ -775,7 +825,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 }
                 if (!ok) break;
             } else {
-                if (!wait_acc()) break;
+                if (!wait_acc(u.kb0)) break;
                 t_acc = t_row();
             }
             // The 32 accumulator values of this warp's local chunk lc, in
@@ -824,12 +874,15 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 const int last = sk_cta_of((tsk + 1) * p.num_kb - 1, p.sk_iters, p.sk_grid);
                 const unsigned others = static_cast<unsigned>(last - first);
                 unsigned* counter = p.counters + tsk;
+                bool own = false;
                 if (u.kb0 == 0) {
-                    if (threadIdx.x == 128) *last_flag = (ld_acquire_u32(counter) == others) ? 1 : 0;
+                    volatile int* lf = last_flag + fsel;
+                    fsel ^= 1;
+                    if (threadIdx.x == 128) *lf = sk_take_own(p, counter, others) ? 1 : 0;
                     __syncwarp();  // named barriers are .aligned: whole warps arrive
                     epilogue_bar_sync();
+                    own = *lf != 0;
                 }
-                const bool own = (u.kb0 == 0) && *last_flag != 0;
                 bool fix = own;
                 if (!own) {
                     // park the partial, column-major inside the tile (element
@@ -855,10 +908,12 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     if constexpr (!kRegAcc) release_acc();
                     __threadfence();
                     epilogue_bar_sync();
-                    if (threadIdx.x == 128) *last_flag = (atomicAdd(counter, 1u) == others) ? 1 : 0;
+                    volatile int* lf = last_flag + fsel;
+                    fsel ^= 1;
+                    if (threadIdx.x == 128) *lf = (atomicAdd(counter, 1u) == others) ? 1 : 0;
                     __syncwarp();
                     epilogue_bar_sync();
-                    fix = *last_flag != 0;
+                    fix = *lf != 0;
                 }
                 if (fix) {
                     __threadfence();
@@ -911,7 +966,10 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     }
 #undef FLE_FIX_BODY
                     epi_finish<SWAP>(p, u, r, best);
-                    if (threadIdx.x == 128) *counter = 0u;
+                    if (threadIdx.x == 128) {
+                        *counter = 0u;
+                        atomicAdd(&g_finish_count[own ? 0 : 1], 1u);
+                    }
                     __syncwarp();
                 }
                 if constexpr (!kRegAcc) {

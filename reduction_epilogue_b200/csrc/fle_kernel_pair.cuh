@@ -28,6 +28,7 @@
 namespace fle {
 
 constexpr int kPairBN = 256;  // pair tile N (B rows), direct operand order
+constexpr int kPairBNNarrow = 224;  // the narrower direct tile (fills uneven waves better)
 constexpr int kPairBM = 256;  // pair tile M (A rows)
 
 // KPS: k-blocks per ring stage, as in Cfg: [A k-blocks | B k-blocks].
@@ -45,14 +46,19 @@ struct PairCfg {
     static constexpr int kEpiStageBytes = kEpiWarps * kEpiTileBytes;
     static constexpr int kStagesRaw = (kSmemStageBudget - kEpiStageBytes) / kStageBytes;
     static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
-    static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
-                                    : (2 * BN <= 256) ? 256 : 512;  // 2 accumulator buffers x BN columns
+    // TMEM columns per accumulator buffer: BN, or 256 for the wide tiles
+    // (BN = 224 keeps its second buffer at column 256)
+    static constexpr int kAccCols = BN > 128 ? 256 : BN;
+    static constexpr int kTmemCols = (2 * kAccCols <= 32) ? 32 : (2 * kAccCols <= 64) ? 64
+                                    : (2 * kAccCols <= 128) ? 128 : (2 * kAccCols <= 256) ? 256 : 512;
     // full, split, empty per stage; accf, acce per buffer; drain; exit
     static constexpr int kNumBars = 3 * kStages + 4 + 2;
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kEpiStageBytes + kNumBars * 8 + 32;
+    static constexpr int kSmemBytes =
+        1024 + kStages * kStageBytes + kEpiStageBytes + kNumBars * 8 + 32 + (kCheckBarriers ? 64 : 0);
     static_assert(kStages >= 2, "need at least two stages");
     static_assert(KPS == 1 || KPS == 2, "one or two k-blocks per stage");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "pair tile N: 32..256, whole 32-column chunks");
+    static_assert(BN % 16 == 0, "MMA N for M = 256 is a multiple of 16");
     static_assert(kBBytes % 1024 == 0, "B halves keep 1024-byte alignment");
     static_assert(kSmemBytes <= 232448, "exceeds 227 KB of shared memory per block");
 };
@@ -76,7 +82,14 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     uint64_t* bars = reinterpret_cast<uint64_t*>(epi_stage + C::kEpiStageBytes);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    // two slots used in turn (see fle_gemm_kernel)
     volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+    // checking build: the work tag of each stage (per CTA) and of each
+    // accumulator buffer (in the leader)
+    volatile uint32_t* stage_tag = reinterpret_cast<volatile uint32_t*>(tmem_slot + 8);
+    volatile uint32_t* acc_tag = stage_tag + 12;
+    (void)stage_tag;
+    (void)acc_tag;
 
     auto bar_full = [&](int s) { return smem_u32(bars + s); };
     auto bar_split = [&](int s) { return smem_u32(bars + S + s); };
@@ -94,6 +107,9 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     const uint32_t rank = cluster_ctarank();  // 0: leader, 1: peer
     const int pair = blockIdx.x >> 1;
     const int num_pairs = gridDim.x >> 1;
+    // The peer's abort flag: a wait that times out raises it too, so that the
+    // other CTA's roles stop waiting for barriers this CTA no longer signals.
+    const uint32_t peer_abort = mapa_shared(smem_u32(const_cast<int*>(abort_flag)), rank ^ 1u);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -138,9 +154,16 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 for (int kb = u.kb0; kb < u.kb1; kb += KPS) {
                     const int n = (u.kb1 - kb < KPS) ? u.kb1 - kb : KPS;  // k-blocks in this stage
                     if (!mbar_wait_bounded(bar_empty(stage), phase ^ 1u, abort_flag, p.timeout_ns,
-                                           kWhereProdEmpty)) {
+                                           kWhereProdEmpty, peer_abort)) {
                         ok = false;
                         break;
+                    }
+                    if constexpr (kCheckBarriers) {
+                        // the full barrier in use: each CTA's own (3xTF32), the leader's (TF32)
+                        if ((k3x || rank == 0) && mbar_test_wait(bar_full(stage), phase))
+                            record_error(kErrProtocol, kWhereProdEmpty);
+                        stage_tag[stage] = work_tag(u.t, kb);
+                        asm volatile("fence.acq_rel.cluster;" ::: "memory");
                     }
                     if constexpr (k3x) {
                         // own barrier: this CTA's split warps wait for these bytes
@@ -168,7 +191,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 const int s = static_cast<int>(f % S);
                 const uint32_t ph = static_cast<uint32_t>((f / S) & 1);
                 volatile int never = 0;
-                mbar_wait_bounded(bar_empty(s), ph, &never, p.timeout_ns, kWhereProdDrain);
+                mbar_wait_bounded(bar_empty(s), ph, &never, kDrainTimeoutNs, kWhereProdDrain);
             }
         }
     } else if (warp == 1) {
@@ -186,20 +209,31 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 for (int kc = u.kb0; ok && kc < u.kb1; kc += kChunkKb) {
                     const int kce = (u.kb1 - kc > kChunkKb) ? kc + kChunkKb : u.kb1;
                     if (!mbar_wait_bounded(bar_acce(buf), acc_phase ^ 1u, abort_flag, p.timeout_ns,
-                                           kWhereMmaAccEmpty)) {
+                                           kWhereMmaAccEmpty, peer_abort)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+                    if constexpr (kCheckBarriers) {
+                        acc_tag[buf] = work_tag(u.t, kc);
+                        asm volatile("fence.acq_rel.cluster;" ::: "memory");
+                    }
+                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * C::kAccCols);
                     for (int kb = kc; kb < kce; kb += KPS) {
                         const int n = (kce - kb < KPS) ? kce - kb : KPS;  // k-blocks in this stage
                         const uint32_t wbar = k3x ? bar_split(stage) : bar_full(stage);
-                        if (!mbar_wait_bounded(wbar, phase, abort_flag, p.timeout_ns, kWhereMmaFull)) {
+                        if (!mbar_wait_bounded(wbar, phase, abort_flag, p.timeout_ns, kWhereMmaFull, peer_abort)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after_sync();
+                        if constexpr (kCheckBarriers) {
+                            // this CTA's stage and the peer's hold the same work
+                            const uint32_t want = work_tag(u.t, kb);
+                            check_tag(stage_tag[stage], want, kWhereMmaFull);
+                            check_tag(ld_cluster_u32(mapa_shared(smem_u32(const_cast<uint32_t*>(stage_tag + stage)), 1)),
+                                      want, kWhereMmaFull);
+                        }
                         auto desc = [](uint32_t a) { return smem_desc_sw128(a); };
                         for (int j = 0; j < n; ++j) {
                             const uint64_t a_hi = desc(sA(stage) + j * C::kABytes);
@@ -231,7 +265,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             }
             mma_commit_pair(bar_drain);
             volatile int never = 0;
-            mbar_wait_bounded(bar_drain, 0, &never, p.timeout_ns, kWhereDrain);
+            mbar_wait_bounded(bar_drain, 0, &never, kDrainTimeoutNs, kWhereDrain);
         }
         __syncwarp();
     } else if (warp < 4) {
@@ -248,9 +282,12 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 for (int kb = u.kb0; kb < u.kb1; kb += KPS) {
                     int got = 0;
                     if (lane == 0)
-                        got = mbar_wait_bounded(bar_full(stage), phase, abort_flag, p.timeout_ns, kWhereConvFull);
+                        got = mbar_wait_bounded(bar_full(stage), phase, abort_flag, p.timeout_ns, kWhereConvFull, peer_abort);
                     got = __shfl_sync(0xffffffffu, got, 0);
                     if (!got) { ok = false; break; }
+                    if constexpr (kCheckBarriers) {
+                        if (lane == 0) check_tag(stage_tag[stage], work_tag(u.t, kb), kWhereConvFull);
+                    }
                     const float4* x4 = reinterpret_cast<const float4*>(smem + stage * C::kStageBytes);
                     float4* lo4 = reinterpret_cast<float4*>(smem + stage * C::kStageBytes + C::kLoadBytes);
                     constexpr int kVec = C::kLoadBytes / 16;
@@ -288,6 +325,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         int buf = 0;
         uint32_t acc_phase = 0;
         float accr[k3x ? kHalf * 32 : 1];  // 3xTF32: this thread's sums of the K slices
+        int fsel = 0;  // next last_flag slot (the same in every epilogue thread)
         Sched sc;
         sc.init(p, pair, num_pairs);
         Unit u;
@@ -300,10 +338,17 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             Unit uh = u;
             uh.ta = 2 * u.ta + static_cast<int>(rank);
             eo.row0 = static_cast<int64_t>(uh.ta) * kBM + q * 32;
-            auto wait_acc = [&]() -> bool {
+            auto wait_acc = [&](int kc) -> bool {
                 int got = 0;
-                if (lane == 0)
-                    got = mbar_wait_bounded(bar_accf(buf), acc_phase, abort_flag, p.timeout_ns, kWhereEpiAccFull);
+                if (lane == 0) {
+                    got = mbar_wait_bounded(bar_accf(buf), acc_phase, abort_flag, p.timeout_ns, kWhereEpiAccFull, peer_abort);
+                    if constexpr (kCheckBarriers) {
+                        // the leader's MMA tagged the buffer it filled
+                        if (got)
+                            check_tag(ld_cluster_u32(mapa_shared(smem_u32(const_cast<uint32_t*>(acc_tag + buf)), 0)),
+                                      work_tag(u.t, kc), kWhereEpiAccFull);
+                    }
+                }
                 got = __shfl_sync(0xffffffffu, got, 0);
                 if (got) tc_fence_after_sync();
                 return got != 0;
@@ -317,7 +362,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 if (buf == 0) acc_phase ^= 1u;
             };
             auto t_row = [&]() {
-                return tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * BN);
+                return tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * C::kAccCols);
             };
 
             uint32_t t_acc = 0;
@@ -325,7 +370,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
 #pragma unroll
                 for (int j = 0; j < kHalf * 32; ++j) accr[j] = 0.0f;
                 for (int kc = u.kb0; kc < u.kb1; kc += kChunkKb) {
-                    if (!wait_acc()) { ok = false; break; }
+                    if (!wait_acc(kc)) { ok = false; break; }
                     const uint32_t tr = t_row();
 #pragma unroll
                     for (int lc = 0; lc < kHalf; ++lc) {
@@ -342,7 +387,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 }
                 if (!ok) break;
             } else {
-                if (!wait_acc()) break;
+                if (!wait_acc(u.kb0)) break;
                 t_acc = t_row();
             }
 
@@ -377,12 +422,15 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 const int last = sk_cta_of((tsk + 1) * p.num_kb - 1, p.sk_iters, p.sk_grid);
                 const unsigned others = static_cast<unsigned>(last - first);
                 unsigned* counter = p.counters + 2 * tsk + rank;
+                bool own = false;
                 if (u.kb0 == 0) {
-                    if (threadIdx.x == 128) *last_flag = (ld_acquire_u32(counter) == others) ? 1 : 0;
+                    volatile int* lf = last_flag + fsel;
+                    fsel ^= 1;
+                    if (threadIdx.x == 128) *lf = sk_take_own(p, counter, others) ? 1 : 0;
                     __syncwarp();  // named barriers are .aligned: whole warps arrive
                     epilogue_bar_sync();
+                    own = *lf != 0;
                 }
-                const bool own = (u.kb0 == 0) && *last_flag != 0;
                 bool fix = own;
                 if (!own) {
                     // park this CTA's partial (column-major: element (row, col)
@@ -410,10 +458,12 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     }
                     __threadfence();
                     epilogue_bar_sync();
-                    if (threadIdx.x == 128) *last_flag = (atomicAdd(counter, 1u) == others) ? 1 : 0;
+                    volatile int* lf = last_flag + fsel;
+                    fsel ^= 1;
+                    if (threadIdx.x == 128) *lf = (atomicAdd(counter, 1u) == others) ? 1 : 0;
                     __syncwarp();
                     epilogue_bar_sync();
-                    fix = *last_flag != 0;
+                    fix = *lf != 0;
                 }
                 if (fix) {
                     __threadfence();
@@ -477,7 +527,10 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                         }
                     }
                     epi_finish<SWAP>(p, uh, r, best);
-                    if (threadIdx.x == 128) *counter = 0u;
+                    if (threadIdx.x == 128) {
+                        *counter = 0u;
+                        atomicAdd(&g_finish_count[own ? 0 : 1], 1u);
+                    }
                     __syncwarp();
                 }
                 if constexpr (!k3x) {
@@ -495,12 +548,14 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     __syncwarp();
     // Neither CTA may release TMEM or exit while the other can still signal
     // its barriers or (leader) write its TMEM: a bounded two-way handshake.
+    // The other CTA arrives within one progress limit (a stalled role gives
+    // up, or sees the abort this CTA raised) plus its drains.
     tc_fence_before_sync();
     __syncthreads();
     if (threadIdx.x == 0) {
         mbar_arrive_cluster(mapa_shared(bar_exit, rank ^ 1u));
         volatile int never = 0;
-        mbar_wait_bounded(bar_exit, 0, &never, p.timeout_ns, kWhereDrain);
+        mbar_wait_bounded(bar_exit, 0, &never, p.timeout_ns + 2 * kDrainTimeoutNs, kWhereDrain);
     }
     __syncwarp();
     __syncthreads();

@@ -15,6 +15,20 @@ namespace fle {
 // ----------------------------------------------------------------------------
 __device__ unsigned int g_status[4];
 
+// How each tile whose k-range was split over CTAs was finished since the
+// counts were last cleared: [0] by the CTA holding k-block 0 from its own
+// accumulator, [1] by the last contributor to arrive, from the parked partials.
+__device__ unsigned int g_finish_count[2];
+
+// Limit of the waits that drain work already issued (tile copies in flight,
+// MMAs not yet complete) before a CTA releases TMEM and exits.  Such work
+// always completes, so this limit is fixed and long, and independent of the
+// progress limit the caller sets (FLE_TIMEOUT_MS).
+constexpr uint64_t kDrainTimeoutNs = 4000000000ull;
+
+// "No peer CTA" for mbar_wait_bounded.
+constexpr uint32_t kNoPeer = 0xFFFFFFFFu;
+
 __device__ __forceinline__ void record_error(unsigned code, unsigned where) {
     if (atomicCAS(&g_status[0], 0u, code) == 0u) {
         g_status[1] = where;
@@ -77,12 +91,69 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// ----------------------------------------------------------------------------
+// Barrier-protocol checks (a build with -DFLE_CHECK_BARRIERS).  The producer
+// of each ring stage and of each TMEM accumulator writes a tag naming the
+// work it holds (tile, first k-block) next to it; every consumer, after its
+// barrier wait, compares that tag with the work its own walk of the schedule
+// expects, and records status 10 (FLE_ERR_PROTOCOL) with the site on a
+// mismatch.  A role that skipped, repeated or reordered a stage or an
+// accumulator, or a parity that aliased a phase, shows up as a wrong tag.
+// Before re-arming a stage the producer also checks, without waiting, that
+// the phase it is about to fill has not already completed.  Without the
+// define all of this compiles away.
+// ----------------------------------------------------------------------------
+#ifdef FLE_CHECK_BARRIERS
+constexpr bool kCheckBarriers = true;
+#else
+constexpr bool kCheckBarriers = false;
+#endif
+constexpr unsigned kErrProtocol = 10u;
+
+__host__ __device__ __forceinline__ uint32_t work_tag(int t, int kb) {
+    return static_cast<uint32_t>(t) * 65537u + static_cast<uint32_t>(kb) + 1u;
+}
+
+// Records a protocol error when the tag at `slot` is not `expect`.
+__device__ __forceinline__ void check_tag(uint32_t got, uint32_t expect, unsigned where) {
+    if (got != expect) record_error(kErrProtocol, where);
+}
+
+// Whether the barrier phase with this parity has completed (no waiting).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// A 32-bit word in shared memory of a CTA of this cluster (address from mapa).
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t remote_addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(remote_addr) : "memory");
+    return v;
+}
+
+// Stores a 32-bit word into shared memory of a CTA of this cluster (address
+// from mapa).
+__device__ __forceinline__ void st_cluster_u32(uint32_t remote_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(remote_addr), "r"(v) : "memory");
+}
+
 // Waits until the barrier phase with the given parity has completed.  Gives
-// up when *abort is set by another role, or after timeout_ns; on a timeout it
-// records FLE_ERR_TIMEOUT (code 8) with `where` and raises *abort.
+// up when *abort is set by another role (of this CTA or of the peer CTA of a
+// pair), or after timeout_ns; on a timeout it records FLE_ERR_TIMEOUT (code 8)
+// with `where` and raises *abort, and also the peer's abort flag when
+// peer_abort (a shared::cluster address) is not kNoPeer, so that the other
+// CTA of a pair stops waiting for signals this one will no longer send.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   volatile int* abort, uint64_t timeout_ns,
-                                                  unsigned where) {
+                                                  unsigned where, uint32_t peer_abort = kNoPeer) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     uint32_t spins = 0;
@@ -92,6 +163,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
         if ((++spins & 31u) == 0u && global_timer_ns() - t0 > timeout_ns) {
             record_error(8u, where);
             *abort = 1;
+            if (peer_abort != kNoPeer) st_cluster_u32(peer_abort, 1u);
             return false;
         }
     }

@@ -47,10 +47,18 @@ def integer_inputs(M: int, K: int, N: int, seed: int = 0, device="cpu", lo: int 
 
 
 def sample_rows(M: int, n: int, seed: int = 0):
-    """A sorted seeded subset of n distinct row indices in [0, M) that always
-    holds the first and last row (tile edges)."""
+    """A sorted seeded subset of exactly min(n, M) distinct row indices in
+    [0, M) that holds the first and last row (tile edges) when n >= 2."""
     n = min(n, M)
+    if n <= 0:
+        return []
+    if n == M:
+        return list(range(M))
     g = _gen(seed + 7919, "cpu")
-    perm = torch.randperm(M, generator=g)[: max(n - 2, 0)].tolist()
-    rows = sorted(set(perm) | {0, M - 1})
-    return rows[:n] if len(rows) > n else rows
+    picked = [0, M - 1][:n]
+    for r in torch.randperm(M, generator=g).tolist():
+        if len(picked) == n:
+            break
+        if r not in (0, M - 1):
+            picked.append(r)
+    return sorted(set(picked))

@@ -34,8 +34,42 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for want in ["fle_forward", "fle_workspace_size", "fle_status_string", "fle_device_status",
-                 "fle_plan_string", "fle_version", "fle_test_bounded_wait"]:
+                 "fle_plan_string", "fle_version", "fle_source_hash", "fle_forward_noalloc",
+                 "fle_test_bounded_wait", "fle_test_epilogue_math", "fle_test_set_finisher",
+                 "fle_test_finisher_counts"]:
         assert want in names
+
+
+def test_test_hooks_live_in_the_testing_header():
+    # the product header declares no test hook; fle_testing.h holds them all
+    inc = os.path.join(ROOT, "include")
+    product = re.sub(r"/\*.*?\*/", "", open(os.path.join(inc, "fle.h")).read(), flags=re.S)
+    testing = re.sub(r"/\*.*?\*/", "", open(os.path.join(inc, "fle_testing.h")).read(), flags=re.S)
+    assert "fle_test_" not in product
+    assert set(re.findall(r"\b(fle_test_\w+)\s*\(", testing)) == {
+        "fle_test_bounded_wait", "fle_test_epilogue_math", "fle_test_set_finisher", "fle_test_finisher_counts"}
+
+
+def test_library_is_built_from_these_sources(lib):
+    # the library carries the hash of the sources and flags it was built from
+    assert lib.fle_source_hash().decode() == fle_build.source_hash()
+    assert not fle_build.needs_build()
+
+
+def test_load_refuses_a_library_of_other_sources(monkeypatch):
+    # a library whose hash does not match the sources beside it is not used
+    monkeypatch.setattr(fle_build, "source_hash", lambda check=False: "0" * 64)
+    monkeypatch.setattr(fle, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built from the sources"):
+        fle.load()
+
+
+def test_finisher_mode_hook_without_a_device(lib):
+    # the mode is host state: set, read back, refuse unknown values
+    assert lib.fle_test_set_finisher(2) == 0
+    assert lib.fle_test_set_finisher(1) == 2
+    assert lib.fle_test_set_finisher(9) == -1
+    assert lib.fle_test_set_finisher(0) == 1
 
 
 def test_library_exports_every_declared_symbol(lib):

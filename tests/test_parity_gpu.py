@@ -6,7 +6,18 @@ Tolerances (elementwise, ref = oracle):
   TF32     |got - ref| <= 5e-3 + 5e-3 |ref|
 Small shapes (several tiles plus ragged tails, both the direct and the
 swapped operand order) are compared in full; the full-size workloads on a
-seeded sample of whole rows, in the same launch plan the benchmark times.
+seeded sample of at least 64 whole rows (every row where M <= 128, and the
+whole [M] output of the pool epilogue), in the same launch plan the
+benchmark times.
+
+Inputs of large magnitude (x ~ N(0, 50^2)) make TF32's operand rounding,
+not the accumulation, the dominant error.  There the single-pass TF32 result
+is checked twice: against the oracle run on the same operands truncated to
+TF32 (what the tensor core multiplies; checked on the device by
+test_tf32_input_conversion_truncates), at the single-pass tolerance, which
+is the tight check; and against the oracle on the exact operands, at that
+tolerance plus the largest change operand truncation can cause, derived per
+element below (a worst case: it holds for every input, so it is loose).
 """
 import ctypes
 import math
@@ -54,6 +65,44 @@ def _assert_close(got, ref, precision, what=""):
                     f"got {got[i]!r} ref {ref[i]!r} err {err[i]:.3e} bound {bound[i]:.3e}")
 
 
+def _tf32(a):
+    """fp32 values with the low 13 mantissa bits cleared: the TF32 operand
+    the tensor core reads for an fp32 input."""
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+    return (a.view(np.uint32) & np.uint32(0xFFFFE000)).view(np.float32)
+
+
+# Largest slope of the exact-form GELU on [-2, 2]: GELU'(t) = Phi(t) + t phi(t)
+# peaks at t = sqrt(2), where it is Phi(sqrt 2) + sqrt(2) phi(sqrt 2) = 1.1289.
+GELU_SLOPE_2 = 1.13
+
+
+def _truncation_bound(x, W, scale):
+    """Per-element bound on how far epilogue (a) can move when both operands
+    are truncated to TF32: each truncation changes a value by less than 2^-10
+    of itself, so a product by less than 2^-9 of |x||W| (to first order),
+    and y by less than 2^-9 sum_k |x_mk| |W_nk|; the clamp is 1-Lipschitz and
+    GELU on [-2, 2] at most 1.13-Lipschitz, after the scale."""
+    ax = np.abs(np.asarray(x.cpu().numpy(), dtype=np.float64))
+    aw = np.abs(np.asarray(W.cpu().numpy(), dtype=np.float64))
+    return GELU_SLOPE_2 * abs(scale) * 2.0 ** -9 * (ax @ aw.T)
+
+
+def _assert_tf32_large_magnitude(got, x, W, b, what):
+    """The two single-pass TF32 checks of large-magnitude inputs (module
+    docstring), for epilogue (a) with the pages' constants."""
+    atol, rtol = TOL["tf32"]
+    got = np.asarray(got, dtype=np.float64)
+    xt, Wt = _tf32(x.cpu().numpy()), _tf32(W.cpu().numpy())
+    ref_t = oracle.forward_rows(xt, Wt, None if b is None else b.cpu().numpy(),
+                                **oracle.PROBLEMS["scale_hardtanh_gelu"])
+    _assert_close(got, ref_t, "tf32", what + " (TF32 operands)")
+    ref = _oracle(x, W, b, "scale_hardtanh_gelu").astype(np.float64)
+    bound = atol + rtol * np.abs(ref) + _truncation_bound(x, W, 0.5)
+    err = np.abs(got - ref)
+    assert (err <= bound).all(), f"{what}: max err {err.max():.3e} outside the derived bound"
+
+
 def _run(fle, x, W, b, problem, precision):
     out = fle.linear_epilogue(x, W, b, problem, precision)
     torch.cuda.synchronize()
@@ -77,13 +126,14 @@ def test_small_full_compare(fle, M, K, N, problem, precision):
     _assert_close(out.cpu().numpy(), _oracle(x, W, b, problem), precision, f"{problem} {M}x{K}x{N}")
 
 
-# Full-size workloads: (M, K, N, problem, sampled rows)
+# Full-size workloads: (M, K, N, problem, sampled rows); at least 64 rows,
+# all rows where M <= 128 and the whole [M] output of the pool epilogue
 FULL = [
     (2048, 8192, 8192, "scale_hardtanh_gelu", 64),
-    (1024, 8192, 8192, "avgpool_gelu_scale_rowmax", 64),
-    (128, 32768, 32768, "swish_scale", 48),
+    (1024, 8192, 8192, "avgpool_gelu_scale_rowmax", 1024),
+    (128, 32768, 32768, "swish_scale", 128),
     (128, 1024, 1024, "scale_hardtanh_gelu", 128),
-] + [(m, 8192, 8192, "scale_hardtanh_gelu", 24) for m in (16, 64, 256, 1024, 4096)]
+] + [(m, 8192, 8192, "scale_hardtanh_gelu", 64) for m in (16, 64, 256, 1024, 4096)]
 
 
 @pytest.mark.parametrize("precision", ["tf32", "3xtf32"])
@@ -92,6 +142,7 @@ def test_full_size_sampled_rows(fle, M, K, N, problem, nrows, precision):
     x, W, b = synth.linear_inputs(M, K, N, seed=0, device="cuda")
     out = _run(fle, x, W, b, problem, precision)
     rows = synth.sample_rows(M, nrows, seed=1)
+    assert len(rows) == min(M, nrows) and len(rows) >= min(M, 64)
     got = out.cpu().numpy()[rows]
     ref = _oracle(x, W, b, problem, rows=rows)
     _assert_close(got, ref, precision, f"{problem} {M}x{K}x{N} rows={len(rows)}")
@@ -114,17 +165,15 @@ def test_integer_inputs_are_exact(fle, M, K, N, precision):
 @pytest.mark.parametrize("M", [64, 512])
 def test_hardtanh_saturation(fle, M, precision):
     # x ~ N(0, 50^2) drives most of 0.5*y past +-2: both clamp branches fire.
-    # The rounding error of a TF32 product scales with the operands, so the
-    # single-pass TF32 bound is the unit-variance one scaled by x's std (50);
-    # 3xTF32 keeps its own bound unchanged.
+    # Single-pass TF32 is checked as the module docstring says; 3xTF32 keeps
+    # its own bound unchanged.
     K, N = 256, 384
     x, W, b = synth.linear_inputs(M, K, N, seed=9, device="cuda", x_std=50.0)
     out = _run(fle, x, W, b, "scale_hardtanh_gelu", precision)
     ref = _oracle(x, W, b, "scale_hardtanh_gelu")
     assert (ref > 1.95).mean() > 0.1 and (ref < -0.045).mean() > 0.1
     if precision == "tf32":
-        err = np.abs(out.cpu().numpy().astype(np.float64) - ref)
-        assert (err <= 50 * (5e-3 + 5e-3 * np.abs(ref))).all(), err.max()
+        _assert_tf32_large_magnitude(out.cpu().numpy(), x, W, b, "saturation")
     else:
         _assert_close(out.cpu().numpy(), ref, precision, "saturation")
 
@@ -415,14 +464,12 @@ def test_fold_scale_option(fle, M, K, N, precision):
         out = fle.linear_epilogue(xin, W, b, "scale_hardtanh_gelu", precision, fold_scale=True)
         torch.cuda.synchronize()
         assert fle.device_status() == 0
-        ref = _oracle(xin, W, b, "scale_hardtanh_gelu")
-        if xin is x:
-            _assert_close(out.cpu().numpy(), ref, precision, f"fold scale {M}x{K}x{N}")
+        if xin is x50 and precision == "tf32":
+            # operand truncation dominates: the checks of the module docstring
+            _assert_tf32_large_magnitude(out.cpu().numpy(), xin, W, b, f"fold scale x50 {M}x{K}x{N}")
         else:
-            # TF32 operand error grows with |x| (x 50): scale the bound likewise
-            atol, rtol = TOL[precision]
-            err = np.abs(out.cpu().numpy().astype(np.float64) - ref)
-            assert (err <= 50 * (atol + rtol * np.abs(ref))).all()
+            ref = _oracle(xin, W, b, "scale_hardtanh_gelu")
+            _assert_close(out.cpu().numpy(), ref, precision, f"fold scale {M}x{K}x{N}")
 
 
 def test_concurrent_calls_on_two_streams(fle):

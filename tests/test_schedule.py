@@ -175,15 +175,44 @@ def test_workspace_matches_the_plan():
     assert g.value == 74  # CTA pairs, whole tiles: no workspace
 
 
+def _tiles(per):
+    return 1 + max(int(r[0]) for rows in per for r in rows)
+
+
+def test_pair_tile_width_fills_the_waves():
+    # Direct pair plans take 224-wide tiles instead of 256 when that fills the
+    # waves on 74 pairs better: 1024 x 8192 x 8192 in TF32 is 4 x 37 = 148
+    # tiles, two full waves with no split (256 wide: 128 tiles, the second
+    # wave 54 of 74 pairs).  In 3xTF32 the 256-wide plan spreads that uneven
+    # wave over all pairs instead, which costs about as much, and it keeps
+    # 256.  256 x 8192 x 8192 is 37 tiles split in two on all 74 pairs (256
+    # wide: 32 tiles on 64 pairs).  The headline 2048 x 8192 x 8192 keeps 256
+    # (3.5 waves of 256 columns = 4 waves of 224).
+    d = fle.desc_for("avgpool_gelu_scale_rowmax", "tf32")
+    grid, per = collect(1024, 8192, 8192, d, 148)
+    assert grid == 74 and _tiles(per) == 148 and all(int(r[5]) == 0 for rows in per for r in rows)
+    d = fle.desc_for("avgpool_gelu_scale_rowmax", "3xtf32")
+    grid, per = collect(1024, 8192, 8192, d, 148)
+    assert grid == 74 and _tiles(per) == 128
+    d = fle.desc_for("scale_hardtanh_gelu", "tf32")
+    grid, per = collect(256, 8192, 8192, d, 148)
+    assert grid == 74 and _tiles(per) == 37
+    assert all(len(rows) == 1 and int(rows[0][5]) == 1 for rows in per)
+    grid, per = collect(2048, 8192, 8192, d, 148)
+    assert _tiles(per) == 8 * 32
+
+
 def test_uneven_last_wave_spreads_only_in_3xtf32():
-    # 1024 x 8192 x 8192 on 74 pairs: 128 tiles = 74 + 54.  The 54 tiles of
-    # the last wave cannot be split evenly (74 // 54 = 1): TF32 runs two whole
-    # waves (CTAs sharing a weight slab keep reading it together from L2),
-    # 3xTF32 spreads the last wave's k-blocks over all 74 pairs.
+    # 512 x 8192 x 14336 on 74 pairs: in TF32, 2 x 64 = 128 tiles of 224 =
+    # 74 + 54.  The 54 tiles of the last wave cannot be split evenly
+    # (74 // 54 = 1): TF32 runs two whole waves (CTAs sharing a weight slab
+    # keep reading it together from L2); 3xTF32 (112 tiles of 256 = 74 + 38)
+    # spreads the last wave's k-blocks over all 74 pairs.
     tf = fle.desc_for("avgpool_gelu_scale_rowmax", "tf32")
-    grid, per = collect(1024, 8192, 8192, tf, 148)
-    assert grid == 74 and all(int(r[5]) == 0 for rows in per for r in rows)
+    grid, per = collect(512, 8192, 14336, tf, 148)
+    assert grid == 74 and _tiles(per) == 128 and all(int(r[5]) == 0 for rows in per for r in rows)
     x3 = fle.desc_for("avgpool_gelu_scale_rowmax", "3xtf32")
-    grid, per = collect(1024, 8192, 8192, x3, 148)
+    grid, per = collect(512, 8192, 14336, x3, 148)
     load = [sum(int(r[4]) - int(r[3]) for r in rows) for rows in per]
-    assert grid == 74 and sum(load) == 128 * 256 and max(load) - min(load) <= 1
+    assert grid == 74 and _tiles(per) == 112
+    assert sum(load) == 112 * 256 and max(load) - min(load) <= 1

@@ -13,8 +13,6 @@ over every SM, and a split last wave) and one that needs none.
 This file is collected last on purpose, and it builds and loads the library
 itself, so it passes alone in a fresh process as well as after the others.
 """
-import ctypes
-
 import numpy as np
 import pytest
 
@@ -74,14 +72,23 @@ def test_noalloc_matches_workspace_entry_point(fle, M, K, N, problem, precision,
         assert (err <= atol + rtol * np.abs(ref)).all(), f"call {call}: max err {err.max():.3e}"
 
 
-def test_noalloc_scratch_bound_covers_every_plan(fle):
-    # The static scratch is 40 MiB; on 148 SMs no plan needs more than
-    # 2 partial tiles of 128 x 256 fp32 per CTA plus counters.
-    assert 2 * 148 * 128 * 256 * 4 + 4096 < 40 << 20
-    lib = fle.load()
-    n = ctypes.c_int(0)
-    g = ctypes.c_int(0)
-    desc = fle.desc_for("scale_hardtanh_gelu", "tf32")
-    assert lib.fle_plan_units(256, 8192, 8192, ctypes.byref(desc), 148, 0, None, 0,
-                              ctypes.byref(n), ctypes.byref(g)) == 0
-    assert fle.workspace_size(256, 8192, 8192, desc) <= 40 << 20
+def test_noalloc_scratch_covers_every_plan(fle):
+    # fle.h states that on a 148-SM B200 no plan needs more than the 40 MiB
+    # static scratch.  Ask the library for the workspace of every benchmark
+    # workload and of seeded random shapes, in both precisions and every
+    # epilogue kind, on this device.
+    import random
+    kinds = ["scale_hardtanh_gelu", "swish_scale", "avgpool_gelu_scale_rowmax", "none"]
+    shapes = [(128, 1024, 1024), (2048, 8192, 8192), (1024, 8192, 8192), (128, 32768, 32768),
+              (16, 8192, 8192), (64, 8192, 8192), (256, 8192, 8192), (1024, 8192, 8192),
+              (4096, 8192, 8192), (65536, 32768, 65536)]
+    rng = random.Random(1234)
+    shapes += [(rng.randint(1, 70000), 4 * rng.randint(1, 16384), rng.randint(16, 70000)) for _ in range(300)]
+    worst = 0
+    for M, K, N in shapes:
+        for problem in kinds:
+            for precision in ("tf32", "3xtf32"):
+                need = fle.workspace_size(M, K, N, fle.desc_for(problem, precision))
+                worst = max(worst, need)
+                assert need <= 40 << 20, (M, K, N, problem, precision, need)
+    assert worst > 0
