@@ -161,6 +161,7 @@ struct Plan {
     int64_t sk_iters = 0;      // k-blocks of the remaining tiles, spread over sk_grid CTAs
     int sk_tiles = 0;
     int sk_grid = 0;
+    int sk_slots = 2;          // partial slots per stream-K CTA: 1 when every CTA holds one shared tile
     int grid = 0;
     size_t partial_bytes = 0;  // workspace: 2 partial tiles per CTA ...
     size_t ws_bytes = 0;       // ... then one arrival counter per stream-K tile
@@ -210,12 +211,12 @@ bool poly_disabled() {
     return off;
 }
 
-// FLE_PAIR_BN=224 or 256 fixes the direct pair tile's width (comparisons).
+// FLE_PAIR_BN=224, 256 or 512 fixes the direct pair tile's width (comparisons).
 int pair_bn_override() {
     static int v = [] {
         const char* e = std::getenv("FLE_PAIR_BN");
         const int n = e ? std::atoi(e) : 0;
-        return (n == fle::kPairBN || n == fle::kPairBNNarrow) ? n : 0;
+        return (n == fle::kPairBN || n == fle::kPairBNNarrow || n == fle::kPairBNWide) ? n : 0;
     }();
     return v;
 }
@@ -276,22 +277,38 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
     if (pl.swap) {
         pl.bn = M <= 32 ? 32 : (M <= 64 ? 64 : 128);
     } else if (pl.pair) {
-        // 256 or 224 B rows per pair tile: the narrower tile when it fills
-        // the waves enough better (time ~ columns per tile x waves; e.g.
-        // 1024 x 8192 x 8192: 128 tiles of 256 = 2 waves on 74 pairs, 148
-        // tiles of 224 = 2 full waves, 12.5% fewer columns per pair)
-        // (in 3xTF32 a 256-wide plan that spreads its uneven last wave over
-        // all pairs measured faster than the two whole waves of 224: 805
-        // against 850 us on 1024 x 8192 x 8192)
+        // 256, 224 or 512 B rows per pair tile.  A plan's time is estimated
+        // as columns per tile x waves on the pairs (plan_waves).
+        // - 224 when it fills the waves enough better: 1024 x 8192 x 8192
+        //   is 128 tiles of 256 = 2 waves on 74 pairs, or 148 tiles of 224
+        //   = 2 full waves, 12.5% fewer columns per pair.  (In 3xTF32 a
+        //   256-wide plan that spreads its uneven last wave over all pairs
+        //   measured faster than the two whole waves of 224: 805 against
+        //   850 us on 1024 x 8192 x 8192.)
+        // - 512 (TF32): two 256-wide MMAs share each A tile, so a column
+        //   costs 0.86 of a 256-wide one (measured per wave: 184 against
+        //   2 x 107 us on 2048 x 8192 x 8192), with one TMEM accumulator and
+        //   512-column partials, whose split last wave costs a quarter wave
+        //   more.  Taken when at least 1.5% faster by this estimate:
+        //   2048, 4096 and 1024 x 8192 x 8192 (measured -1.1%, -2.2%, -3.5%);
+        //   not 256 x 8192 x 8192 (16 tiles split four ways: slower).
         const int64_t ta = (M + fle::kPairBM - 1) / fle::kPairBM;
         const int64_t G = pairs;
         const bool spread = pl.prec == fle::kPrec3xTF32;
-        const double c256 = fle::kPairBN *
-                            plan_waves(ta * ((N + fle::kPairBN - 1) / fle::kPairBN), G, num_kb, min_iters, spread);
-        const double c224 = fle::kPairBNNarrow *
-                            plan_waves(ta * ((N + fle::kPairBNNarrow - 1) / fle::kPairBNNarrow), G, num_kb, min_iters, spread);
+        auto tiles_of = [&](int bn) { return ta * ((N + bn - 1) / bn); };
+        const double c256 = fle::kPairBN * plan_waves(tiles_of(fle::kPairBN), G, num_kb, min_iters, spread);
+        const double c224 =
+            fle::kPairBNNarrow * plan_waves(tiles_of(fle::kPairBNNarrow), G, num_kb, min_iters, spread);
         pl.bn = (c224 < 0.97 * c256) ? fle::kPairBNNarrow : fle::kPairBN;
+        if (pl.prec == fle::kPrecTF32) {
+            const int64_t Tw = tiles_of(fle::kPairBNWide);
+            double ww = plan_waves(Tw, G, num_kb, min_iters, false);
+            if (Tw % G != 0 && ww != std::floor(ww)) ww += 0.25;  // split last wave of wide partials
+            const double c512 = 0.86 * fle::kPairBNWide * ww;
+            if (c512 < 0.985 * std::min(c256, c224)) pl.bn = fle::kPairBNWide;
+        }
         if (pair_bn_override() != 0) pl.bn = pair_bn_override();
+        if (pl.bn > 256 && pl.prec != fle::kPrecTF32) pl.bn = fle::kPairBN;  // wide tiles: TF32 only
     } else {
         pl.bn = (pl.prec == fle::kPrec3xTF32) ? 128 : 256;
     }
@@ -310,6 +327,7 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
         const int64_t tiles = static_cast<int64_t>(pl.tiles_a) * pl.tiles_b;
         if (pl.swap || (pl.pair && tiles >= 2 * static_cast<int64_t>(pairs))) pl.kps = 2;
         if (kps_override() != 0) pl.kps = kps_override();
+        if (pl.bn > 256) pl.kps = 1;  // a 512-wide stage of one k-block is already 48 KB
     }
     pl.stages = pl.pair ? pair_stages_for(pl.bn, pl.prec, pl.kps) : stages_for(pl.bn, pl.prec, pl.kps);
 
@@ -363,11 +381,22 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
     pl.sk_tiles = static_cast<int>(T - pl.dp_tiles);
     pl.sk_iters = static_cast<int64_t>(pl.sk_tiles) * pl.num_kb;
     if (pl.sk_tiles > 0) {
-        // two fp32 partial tiles of 128 x bn per stream-K CTA, then one
+        // one partial slot per CTA unless some CTA's stream-K range reaches
+        // into a second tile (the k-aligned split of a last wave never does)
+        pl.sk_slots = 1;
+        for (int64_t c = 0; c < pl.sk_grid; ++c) {
+            const int64_t gb = c * pl.sk_iters / pl.sk_grid;
+            const int64_t ge = (c + 1) * pl.sk_iters / pl.sk_grid;
+            if (ge > gb && gb / pl.num_kb != (ge - 1) / pl.num_kb) {
+                pl.sk_slots = 2;
+                break;
+            }
+        }
+        // sk_slots fp32 partial tiles of 128 x bn per stream-K CTA, then one
         // arrival counter per stream-K tile (per CTA of the pair)
         const int sk_ctas = pl.pair ? 2 * pl.sk_grid : pl.sk_grid;
         const int counters = pl.pair ? 2 * pl.sk_tiles : pl.sk_tiles;
-        pl.partial_bytes = static_cast<size_t>(2) * sk_ctas * fle::kBM * pl.bn * sizeof(float);
+        pl.partial_bytes = static_cast<size_t>(pl.sk_slots) * sk_ctas * fle::kBM * pl.bn * sizeof(float);
         pl.ws_bytes = pl.partial_bytes + ((static_cast<size_t>(counters) * 4 + 255) & ~size_t(255));
     }
     return pl;
@@ -441,6 +470,8 @@ cudaError_t dispatch(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& t
     using namespace fle;
     const bool tf32 = pl.prec == kPrecTF32;
     const bool two = pl.kps == 2;  // TF32 only
+    if (pl.pair && !pl.swap && pl.bn == kPairBNWide)
+        return launch_gemm_pair<kPrecTF32, 1, kPairBNWide>(ta, tb, to, p, pl.grid, after_prep, st);
     if (pl.pair && !pl.swap && pl.bn == kPairBNNarrow) {
         if (!tf32) return launch_gemm_pair<kPrec3xTF32, 1, kPairBNNarrow>(ta, tb, to, p, pl.grid, after_prep, st);
         return two ? launch_gemm_pair<kPrecTF32, 2, kPairBNNarrow>(ta, tb, to, p, pl.grid, after_prep, st)
@@ -522,11 +553,11 @@ int plan_to_string(const Plan& pl, char* buf, size_t n) {
     if (!buf || n == 0) return FLE_ERR_NULL;
     std::snprintf(buf, n,
                   "tile=%dx%d pair=%d swap=%d prec=%s stages=%d kps=%d tiles=%dx%d kblocks=%d dp_tiles=%d sk_tiles=%d "
-                  "sk_kblocks=%lld sk_grid=%d grid=%d workspace=%zu",
+                  "sk_kblocks=%lld sk_grid=%d slots=%d grid=%d workspace=%zu",
                   pl.pair ? fle::kPairBM : fle::kBM, pl.bn, pl.pair ? 1 : 0, pl.swap ? 1 : 0,
                   pl.prec == fle::kPrecTF32 ? "tf32" : "3xtf32", pl.stages, pl.kps,
-                  pl.tiles_a, pl.tiles_b, pl.num_kb, pl.dp_tiles, pl.sk_tiles, (long long)pl.sk_iters, pl.sk_grid, pl.grid,
-                  pl.ws_bytes);
+                  pl.tiles_a, pl.tiles_b, pl.num_kb, pl.dp_tiles, pl.sk_tiles, (long long)pl.sk_iters, pl.sk_grid,
+                  pl.sk_slots, pl.grid, pl.ws_bytes);
     return FLE_OK;
 }
 
@@ -648,6 +679,7 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
     p.dp_tiles = pl.dp_tiles;
     p.sk_iters = pl.sk_iters;
     p.sk_grid = pl.sk_grid;
+    p.sk_slots = pl.sk_slots;
     if (pl.sk_tiles > 0) {
         p.ws = static_cast<float*>(workspace);
         p.counters = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + pl.partial_bytes);
@@ -666,7 +698,9 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
     const float* B = pl.swap ? x : W;
     st = encode_operand(&ta, A, p.Ma, K, fle::kBM);
     if (st != FLE_OK) return st;
-    st = encode_operand(&tb, B, p.Nb, K, pl.pair ? pl.bn / 2 : pl.bn);
+    // B boxes: half of the pair tile's rows per CTA, 128 for the 512-wide
+    // tile (each CTA loads its 128 rows of both 256-wide sub-tiles)
+    st = encode_operand(&tb, B, p.Nb, K, pl.pair ? (pl.bn > 256 ? 128 : pl.bn / 2) : pl.bn);
     if (st != FLE_OK) return st;
 
     if (log_enabled()) {
@@ -711,6 +745,7 @@ int fle_plan_units(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, 
     p.dp_tiles = pl.dp_tiles;
     p.sk_iters = pl.sk_iters;
     p.sk_grid = pl.sk_grid;
+    p.sk_slots = pl.sk_slots;
     fle::Sched sc;
     sc.init(p, cta, pl.grid);
     fle::Unit u;

@@ -57,7 +57,7 @@ enum : unsigned {
 struct KParams {
     const float* bias;      // [N] or nullptr
     float* out;             // [M,N] or [M]
-    float* ws;              // stream-K partial tiles: [2 * grid][kBM * BN]
+    float* ws;              // stream-K partial tiles: [sk_slots * CTAs][kBM * BN]
     unsigned* counters;     // stream-K arrival counters, one per stream-K tile
     int64_t M, N;           // output sizes
     int Ma, Nb;             // rows of operand A and operand B
@@ -67,6 +67,7 @@ struct KParams {
     int dp_tiles;           // tiles [0, dp_tiles) are data-parallel
     int64_t sk_iters;       // (num_tiles - dp_tiles) * num_kb
     int sk_grid;            // CTAs [0, sk_grid) share the stream-K k-blocks
+    int sk_slots;           // partial-tile slots per stream-K CTA (1 or 2)
     int kind;
     float scale, clamp_lo, clamp_hi;
     int gelu_tanh;          // GELU in its tanh form, (a) and (c)
@@ -888,7 +889,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     // park the partial, column-major inside the tile (element
                     // (row, col) at col * 128 + row: a warp's lanes write 32
                     // consecutive floats), then count it
-                    float* slot = p.ws + static_cast<size_t>(2 * blockIdx.x + u.slot) * kBM * BN;
+                    float* slot = p.ws + static_cast<size_t>(p.sk_slots * blockIdx.x + u.slot) * kBM * BN;
 #define FLE_PARK_BODY(lc)                                                                 \
     {                                                                                     \
         float v[32];                                                                      \
@@ -920,7 +921,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     float best = -INFINITY;
                     auto src_of = [&](int cc, int c) {
                         const int sl = sk_slot_of(cc, tsk, p.sk_iters, p.sk_grid, p.num_kb);
-                        return p.ws + static_cast<size_t>(2 * cc + sl) * kBM * BN +
+                        return p.ws + static_cast<size_t>(p.sk_slots * cc + sl) * kBM * BN +
                                static_cast<size_t>(c * 32) * kBM + r;
                     };
                     // start from the own accumulator (contributors first+1 ..

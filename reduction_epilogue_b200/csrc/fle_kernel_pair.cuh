@@ -29,6 +29,7 @@ namespace fle {
 
 constexpr int kPairBN = 256;  // pair tile N (B rows), direct operand order
 constexpr int kPairBNNarrow = 224;  // the narrower direct tile (fills uneven waves better)
+constexpr int kPairBNWide = 512;    // two 256-wide MMAs sharing the A tile (TF32)
 constexpr int kPairBM = 256;  // pair tile M (A rows)
 
 // KPS: k-blocks per ring stage, as in Cfg: [A k-blocks | B k-blocks].
@@ -39,6 +40,11 @@ struct PairCfg {
     static constexpr int kBKW = kBK;  // k-block width: 32 fp32, one 128-byte swizzle row
     static constexpr int kABytes = kBM * kBKW * 4;            // this CTA's 128 A rows, one k-block
     static constexpr int kBBytes = (BN / 2) * kBKW * 4;       // this CTA's BN / 2 B rows, one k-block
+    // Tiles wider than 256 are kNSub MMAs of N = kSubN sharing the A tile;
+    // each CTA holds its kSubN / 2 rows of every sub-tile, one after another.
+    static constexpr int kNSub = BN > 256 ? BN / 256 : 1;
+    static constexpr int kSubN = BN / kNSub;
+    static constexpr int kSubBBytes = kBBytes / kNSub;
     static constexpr int kKbBytes = kABytes + kBBytes;
     static constexpr int kLoadBytes = KPS * kKbBytes;         // TMA bytes per full stage and CTA
     static constexpr int kStageBytes = kLoadBytes * (PREC == kPrec3xTF32 ? 2 : 1);
@@ -46,18 +52,25 @@ struct PairCfg {
     static constexpr int kEpiStageBytes = kEpiWarps * kEpiTileBytes;
     static constexpr int kStagesRaw = (kSmemStageBudget - kEpiStageBytes) / kStageBytes;
     static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
-    // TMEM columns per accumulator buffer: BN, or 256 for the wide tiles
-    // (BN = 224 keeps its second buffer at column 256)
-    static constexpr int kAccCols = BN > 128 ? 256 : BN;
-    static constexpr int kTmemCols = (2 * kAccCols <= 32) ? 32 : (2 * kAccCols <= 64) ? 64
-                                    : (2 * kAccCols <= 128) ? 128 : (2 * kAccCols <= 256) ? 256 : 512;
+    // TMEM accumulator buffers and columns per buffer: two of BN, or of 256
+    // for BN = 224 (its second buffer starts at column 256); one of 512 for
+    // the 512-wide tile, which fills the whole TMEM
+    static constexpr int kNumAcc = BN > 256 ? 1 : 2;
+    static constexpr int kAccCols = BN > 256 ? BN : (BN > 128 ? 256 : BN);
+    static constexpr int kTmemAll = kNumAcc * kAccCols;
+    static constexpr int kTmemCols = (kTmemAll <= 32) ? 32 : (kTmemAll <= 64) ? 64
+                                    : (kTmemAll <= 128) ? 128 : (kTmemAll <= 256) ? 256 : 512;
     // full, split, empty per stage; accf, acce per buffer; drain; exit
     static constexpr int kNumBars = 3 * kStages + 4 + 2;
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kEpiStageBytes + kNumBars * 8 + 32;
     static_assert(kStages >= 2, "need at least two stages");
     static_assert(KPS == 1 || KPS == 2, "one or two k-blocks per stage");
-    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "pair tile N: 32..256, whole 32-column chunks");
-    static_assert(BN % 16 == 0, "MMA N for M = 256 is a multiple of 16");
+    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 512, "pair tile N: 32..512, whole 32-column chunks");
+    static_assert(kSubN % 16 == 0 && kSubN <= 256, "MMA N for M = 256 is a multiple of 16, at most 256");
+    static_assert(BN <= 256 || (BN % 256 == 0 && PREC == kPrecTF32 && !SWAP),
+                  "wide tiles: whole 256-column sub-tiles, single-pass TF32, direct operand order");
+    static_assert(kSubBBytes % 1024 == 0, "B sub-tiles keep 1024-byte alignment");
+    static_assert(kTmemAll <= 512, "TMEM has 512 columns");
     static_assert(kBBytes % 1024 == 0, "B halves keep 1024-byte alignment");
     static_assert(kSmemBytes <= 232448, "exceeds 227 KB of shared memory per block");
 };
@@ -69,7 +82,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     using C = PairCfg<PREC, KPS, BN, SWAP>;
     constexpr bool k3x = (PREC == kPrec3xTF32);
     constexpr int S = C::kStages;
-    constexpr uint32_t kIdesc = idesc_tf32(kPairBM, BN);
+    constexpr uint32_t kIdesc = idesc_tf32(kPairBM, C::kSubN);
     constexpr int kBKW = C::kBKW;
     constexpr int kChunkKb = k3x ? 128 / kBKW : (1 << 30);  // k-blocks per TMEM accumulation chain
     static_assert(kChunkKb % KPS == 0, "accumulation chains hold whole stages");
@@ -143,7 +156,8 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             Unit u;
             while (ok && sc.next(p, u)) {
                 const int32_t ra = u.ta * kPairBM + static_cast<int32_t>(rank) * kBM;
-                const int32_t rb = u.tb * BN + static_cast<int32_t>(rank) * (BN / 2);
+                // B rows of sub-tile s: u.tb * BN + s * kSubN + rank * kSubN / 2, kSubN / 2 of them
+                const int32_t rb = u.tb * BN + static_cast<int32_t>(rank) * (C::kSubN / 2);
                 for (int kb = u.kb0; kb < u.kb1; kb += KPS) {
                     const int n = (u.kb1 - kb < KPS) ? u.kb1 - kb : KPS;  // k-blocks in this stage
                     if (!mbar_wait_bounded(bar_empty(stage), phase ^ 1u, abort_flag, p.timeout_ns,
@@ -156,7 +170,10 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                         mbar_arrive_expect_tx(bar_full(stage), n * C::kKbBytes);
                         for (int j = 0; j < n; ++j) {
                             tma_load_2d(sA(stage) + j * C::kABytes, &tmA, bar_full(stage), (kb + j) * kBKW, ra);
-                            tma_load_2d(sB(stage) + j * C::kBBytes, &tmB, bar_full(stage), (kb + j) * kBKW, rb);
+#pragma unroll
+                            for (int sb = 0; sb < C::kNSub; ++sb)
+                                tma_load_2d(sB(stage) + j * C::kBBytes + sb * C::kSubBBytes, &tmB, bar_full(stage),
+                                            (kb + j) * kBKW, rb + sb * C::kSubN);
                         }
                     } else {
                         // the leader expects both CTAs' bytes on its own full barrier
@@ -164,7 +181,10 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                         const uint32_t leader_full = mapa_shared(bar_full(stage), 0);
                         for (int j = 0; j < n; ++j) {
                             tma_load_2d_pair(sA(stage) + j * C::kABytes, &tmA, leader_full, (kb + j) * kBKW, ra);
-                            tma_load_2d_pair(sB(stage) + j * C::kBBytes, &tmB, leader_full, (kb + j) * kBKW, rb);
+#pragma unroll
+                            for (int sb = 0; sb < C::kNSub; ++sb)
+                                tma_load_2d_pair(sB(stage) + j * C::kBBytes + sb * C::kSubBBytes, &tmB, leader_full,
+                                                 (kb + j) * kBKW, rb + sb * C::kSubN);
                         }
                     }
                     ++fills;
@@ -225,7 +245,11 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                                     mma_tf32_pair(d_tmem, a_hi + koff, b_lo + koff, kIdesc, 1u);
                                     mma_tf32_pair(d_tmem, a_hi + koff, b_hi + koff, kIdesc, 1u);
                                 } else {
-                                    mma_tf32_pair(d_tmem, a_hi + koff, b_hi + koff, kIdesc, acc);
+#pragma unroll
+                                    for (int sb = 0; sb < C::kNSub; ++sb)
+                                        mma_tf32_pair(d_tmem + static_cast<uint32_t>(sb * C::kSubN), a_hi + koff,
+                                                      desc(sB(stage) + j * C::kBBytes + sb * C::kSubBBytes) + koff,
+                                                      kIdesc, acc);
                                 }
                             }
                         }
@@ -234,8 +258,10 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     }
                     if (!ok) break;
                     mma_commit_pair_multicast(bar_accf(buf), 0x3);
-                    buf ^= 1;
-                    if (buf == 0) acc_phase ^= 1u;
+                    if (++buf == C::kNumAcc) {
+                        buf = 0;
+                        acc_phase ^= 1u;
+                    }
                 }
             }
             mma_commit_pair(bar_drain);
@@ -323,8 +349,10 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(mapa_shared(bar_acce(buf), 0));
                 __syncwarp();
-                buf ^= 1;
-                if (buf == 0) acc_phase ^= 1u;
+                if (++buf == C::kNumAcc) {
+                    buf = 0;
+                    acc_phase ^= 1u;
+                }
             };
             auto t_row = [&]() {
                 return tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * C::kAccCols);
@@ -400,7 +428,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 if (!own) {
                     // park this CTA's partial (column-major: element (row, col)
                     // at col * 128 + row) and count it
-                    float* slot = p.ws + static_cast<size_t>(2 * blockIdx.x + u.slot) * kBM * BN;
+                    float* slot = p.ws + static_cast<size_t>(p.sk_slots * blockIdx.x + u.slot) * kBM * BN;
                     if constexpr (k3x) {
 #pragma unroll
                         for (int lc = 0; lc < kHalf; ++lc) {
@@ -435,7 +463,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     float best = -INFINITY;
                     auto src_of = [&](int cc, int c) {
                         const int sl = sk_slot_of(cc, tsk, p.sk_iters, p.sk_grid, p.num_kb);
-                        return p.ws + static_cast<size_t>(2 * (2 * cc + rank) + sl) * kBM * BN +
+                        return p.ws + static_cast<size_t>(p.sk_slots * (2 * cc + rank) + sl) * kBM * BN +
                                static_cast<size_t>(c * 32) * kBM + r;
                     };
                     // contributors from..last added in order; loads of up to

@@ -118,23 +118,37 @@ def check_schedule(M, K, N, problem, precision, sms):
     assert max(load) - min(load) <= num_kb
 
 
-def test_headline_shape_splits_only_the_last_wave():
-    # 2048x8192x8192 in TF32 runs 256x256 tiles on CTA pairs: 256 tiles on the
-    # 74 pairs of 148 SMs is 3.46 waves.  Three waves run whole tiles; the 34
-    # tiles of the last wave are split in two k-aligned halves on 68 pairs, so
-    # the pairs finish within half a tile.
+def test_headline_shape_plans():
+    # 2048x8192x8192 in TF32 runs 256x512 tiles on CTA pairs (two 256-wide
+    # MMAs sharing each x tile): 128 tiles on the 74 pairs of 148 SMs, two
+    # waves of whole tiles.  In 3xTF32 (no wide tiles) it runs 256x256 tiles:
+    # 3.46 waves, three of whole tiles and the 34 tiles of the last wave split
+    # in two k-aligned halves on 68 pairs.
     desc = fle.desc_for("scale_hardtanh_gelu", "tf32")
     grid, per_cta = collect(2048, 8192, 8192, desc, 148)
-    assert grid == 74
+    assert grid == 74 and _tiles(per_cta) == 128
+    assert all(int(r[5]) == 0 for rows in per_cta for r in rows)
     load = [sum(int(r[4]) - int(r[3]) for r in rows) for rows in per_cta]
-    assert sum(load) == 256 * 256
-    assert max(load) - min(load) == 128
-    halves = [r for rows in per_cta for r in rows if r[5]]
+    assert sum(load) == 128 * 256 and sorted(set(load)) == [256, 512]
+    grid3, per3 = collect(2048, 8192, 8192, fle.desc_for("scale_hardtanh_gelu", "3xtf32"), 148)
+    assert grid3 == 74 and _tiles(per3) == 256
+    load = [sum(int(r[4]) - int(r[3]) for r in rows) for rows in per3]
+    assert sum(load) == 256 * 256 and max(load) - min(load) == 128
+    halves = [r for rows in per3 for r in rows if r[5]]
     assert len(halves) == 68
     assert {(int(r[3]), int(r[4])) for r in halves} == {(0, 128), (128, 256)}
-    # 3xTF32 runs the same 256x256 pair tiles (and the same schedule)
-    grid3, per3 = collect(2048, 8192, 8192, fle.desc_for("scale_hardtanh_gelu", "3xtf32"), 148)
-    assert grid3 == 74 and sum(int(r[4]) - int(r[3]) for rows in per3 for r in rows) == 256 * 256
+
+
+def test_k_aligned_split_needs_one_partial_slot():
+    # 4096x8192x8192 in TF32: 256 wide tiles = 3 waves + 34 tiles split in two
+    # k-aligned halves; every CTA holds at most one shared tile, in slot 0, so
+    # the workspace holds one 128x512 partial per stream-K CTA.
+    desc = fle.desc_for("scale_hardtanh_gelu", "tf32")
+    grid, per = collect(4096, 8192, 8192, desc, 148)
+    assert grid == 74 and _tiles(per) == 256
+    shared = [[r for r in rows if int(r[5])] for rows in per]
+    assert sum(len(x) for x in shared) == 68
+    assert all(len(x) <= 1 and all(int(r[6]) == 0 for r in x) for x in shared)
 
 
 def test_weight_streamed_once_shapes_split_each_tile():
@@ -181,16 +195,16 @@ def _tiles(per):
 
 def test_pair_tile_width_fills_the_waves():
     # Direct pair plans take 224-wide tiles instead of 256 when that fills the
-    # waves on 74 pairs better: 1024 x 8192 x 8192 in TF32 is 4 x 37 = 148
-    # tiles, two full waves with no split (256 wide: 128 tiles, the second
-    # wave 54 of 74 pairs).  In 3xTF32 the 256-wide plan spreads that uneven
-    # wave over all pairs instead, which costs about as much, and it keeps
-    # 256.  256 x 8192 x 8192 is 37 tiles split in two on all 74 pairs (256
-    # wide: 32 tiles on 64 pairs).  The headline 2048 x 8192 x 8192 keeps 256
-    # (3.5 waves of 256 columns = 4 waves of 224).
+    # waves on 74 pairs better, and 512-wide tiles (TF32) when those are
+    # enough cheaper per column.  1024 x 8192 x 8192 in TF32: 4 x 16 = 64
+    # tiles of 512, one wave (224 wide: 148 tiles, two full waves; 256 wide:
+    # 128 tiles, the second wave 54 of 74 pairs).  In 3xTF32 (no wide tiles)
+    # the 256-wide plan spreads its uneven wave over all pairs, which costs
+    # about as much as 224, and it keeps 256.  256 x 8192 x 8192 is 37 tiles
+    # of 224 split in two on all 74 pairs (256 wide: 32 tiles on 64 pairs).
     d = fle.desc_for("avgpool_gelu_scale_rowmax", "tf32")
     grid, per = collect(1024, 8192, 8192, d, 148)
-    assert grid == 74 and _tiles(per) == 148 and all(int(r[5]) == 0 for rows in per for r in rows)
+    assert grid == 64 and _tiles(per) == 64 and all(int(r[5]) == 0 for rows in per for r in rows)
     d = fle.desc_for("avgpool_gelu_scale_rowmax", "3xtf32")
     grid, per = collect(1024, 8192, 8192, d, 148)
     assert grid == 74 and _tiles(per) == 128
@@ -199,18 +213,18 @@ def test_pair_tile_width_fills_the_waves():
     assert grid == 74 and _tiles(per) == 37
     assert all(len(rows) == 1 and int(rows[0][5]) == 1 for rows in per)
     grid, per = collect(2048, 8192, 8192, d, 148)
-    assert _tiles(per) == 8 * 32
+    assert _tiles(per) == 8 * 16
 
 
 def test_uneven_last_wave_spreads_only_in_3xtf32():
-    # 512 x 8192 x 14336 on 74 pairs: in TF32, 2 x 64 = 128 tiles of 224 =
-    # 74 + 54.  The 54 tiles of the last wave cannot be split evenly
-    # (74 // 54 = 1): TF32 runs two whole waves (CTAs sharing a weight slab
-    # keep reading it together from L2); 3xTF32 (112 tiles of 256 = 74 + 38)
-    # spreads the last wave's k-blocks over all 74 pairs.
+    # 512 x 8192 x 14336 on 74 pairs.  TF32 runs whole tiles only (2 x 28 =
+    # 56 tiles of 512, one wave; CTAs sharing a weight slab keep reading it
+    # together from L2).  3xTF32 (112 tiles of 256 = 74 + 38; the 38 of the
+    # last wave cannot be split evenly, 74 // 38 = 1) spreads the last wave's
+    # k-blocks over all 74 pairs.
     tf = fle.desc_for("avgpool_gelu_scale_rowmax", "tf32")
     grid, per = collect(512, 8192, 14336, tf, 148)
-    assert grid == 74 and _tiles(per) == 128 and all(int(r[5]) == 0 for rows in per for r in rows)
+    assert grid == 56 and _tiles(per) == 56 and all(int(r[5]) == 0 for rows in per for r in rows)
     x3 = fle.desc_for("avgpool_gelu_scale_rowmax", "3xtf32")
     grid, per = collect(512, 8192, 14336, x3, 148)
     load = [sum(int(r[4]) - int(r[3]) for r in rows) for rows in per]
