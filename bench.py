@@ -295,6 +295,104 @@ def roofline(flops, nbytes, step_ms, precision, name):
     return roof
 
 
+def e2e_serial(x, W, b, out, step, variant, steps, stream, world, dev):
+    """Upload the step's inputs from pinned host memory, run the call, read
+    the result back; the next step starts after the read-back."""
+    import torch
+    xh = x.cpu().pin_memory()
+    Wh = W.cpu().pin_memory()
+    bh = b.cpu().pin_memory()
+    outh = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    copy_w = variant != "poolfold_cached"  # cached pooled weights stay on the device
+
+    def h2d():
+        x.copy_(xh, non_blocking=True)
+        if copy_w:
+            W.copy_(Wh, non_blocking=True)
+            b.copy_(bh, non_blocking=True)
+
+    for _ in range(2):
+        h2d()
+        step()
+        outh.copy_(out, non_blocking=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        h2d()
+        step()
+        outh.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return max_over_ranks(e0.elapsed_time(e1), world, dev), copy_w
+
+
+def e2e_pipelined(fle, desc, bufs, ws, ws_bytes, steps, stream, world, dev):
+    """Every step uploads its inputs (x, W, b) from pinned host memory, runs
+    fle_forward and reads its result back to pinned host memory, with two
+    sets of device buffers: step i+1's upload (copy stream) overlaps step i's
+    kernel (the caller's stream) and step i-1's read-back (a second copy
+    stream).  Events order each buffer set's reuse: an upload waits for the
+    kernel that last read the set, a kernel for the read-back that last read
+    its output.  Returns the time from the first upload to the last
+    read-back, max over ranks."""
+    import torch
+    x, W, b, out = bufs
+    sets = [(x, W, b, out), tuple(torch.empty_like(t) for t in (x, W, b, out))]
+    hosts = [t.cpu().pin_memory() for t in (x, W, b)]
+    outh = [torch.empty(out.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    done_kernel = [None, None]
+    done_read = [None, None]
+
+    def one(i):
+        sidx = i % 2
+        xd, Wd, bd, od = sets[sidx]
+        with torch.cuda.stream(up):
+            if done_kernel[sidx] is not None:
+                up.wait_event(done_kernel[sidx])
+            for dst, src in zip((xd, Wd, bd), hosts):
+                dst.copy_(src, non_blocking=True)
+            uploaded = ev()
+            uploaded.record(up)
+        stream.wait_event(uploaded)
+        if done_read[sidx] is not None:
+            stream.wait_event(done_read[sidx])
+        fle.forward(xd, Wd, bd, od, desc, workspace=ws, workspace_bytes=ws_bytes, stream=stream)
+        done_kernel[sidx] = ev()
+        done_kernel[sidx].record(stream)
+        with torch.cuda.stream(down):
+            down.wait_event(done_kernel[sidx])
+            outh[sidx].copy_(od, non_blocking=True)
+            done_read[sidx] = ev()
+            done_read[sidx].record(down)
+
+    for i in range(2):
+        one(i)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    done_kernel = [None, None]
+    done_read = [None, None]
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(up)
+    for i in range(steps):
+        one(i)
+    for r in done_read:
+        if r is not None:
+            stream.wait_event(r)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    del sets[1]
+    return max_over_ranks(ms, world, dev)
+
+
 def run_fle(args, name, dist_ctx, precision=None, brief=False):
     """Times one workload.  Returns (on rank 0) the JSON line's dict, or with
     brief=True a compact per-config record (no end-to-end, CPU or torch legs)."""
@@ -413,42 +511,22 @@ def run_fle(args, name, dist_ctx, precision=None, brief=False):
             rec["frac_of_3pass"] = roof["frac_of_3pass"]
         return rec
 
-    # end to end through the public call: pinned host inputs in, result out
+    # end to end through the public call: pinned host inputs in, result out,
+    # every step
     e2e = None
     if not args.no_e2e:
-        xh = x.cpu().pin_memory()
-        Wh = W.cpu().pin_memory()
-        bh = b.cpu().pin_memory()
-        outh = torch.empty(out.shape, dtype=torch.float32).pin_memory()
         e2e_steps = max(1, min(steps, args.e2e_steps))
-        copy_w = variant != "poolfold_cached"  # cached pooled weights stay on the device
-
-        def h2d():
-            x.copy_(xh, non_blocking=True)
-            if copy_w:
-                W.copy_(Wh, non_blocking=True)
-                b.copy_(bh, non_blocking=True)
-
-        for _ in range(2):
-            h2d()
-            step()
-            outh.copy_(out, non_blocking=True)
-        if world > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            h2d()
-            step()
-            outh.copy_(out, non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        if variant is None:
+            e_ms = e2e_pipelined(fle, desc, (x, W, b, out), ws, ws_bytes, e2e_steps, stream, world, dev)
+            mode = ("pipelined: two device buffer sets; step i+1's upload overlaps step i's kernel and "
+                    "read-back (one copy stream each way)")
+            copy_w = True
+        else:
+            e_ms, copy_w = e2e_serial(x, W, b, out, step, variant, e2e_steps, stream, world, dev)
+            mode = "serial: upload, kernel, read-back"
         e2e = {"value": job_throughput_tflops(flops, world, e2e_steps, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": (4 * (M * K + N * K + N) if copy_w else 4 * M * K),
-               "d2h_bytes_per_step": 4 * out_elems, "steps": e2e_steps}
+               "d2h_bytes_per_step": 4 * out_elems, "steps": e2e_steps, "mode": mode}
 
     if warm_ms is not None:
         roof["kernel_us_warm_l2"] = warm_ms * 1e3
