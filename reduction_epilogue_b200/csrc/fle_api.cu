@@ -363,10 +363,11 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
             const int64_t S = std::min<int64_t>(G / R, pl.num_kb / min_iters);
             // When the last wave cannot be split evenly (S < 2), 3xTF32 spreads
             // its k-blocks over all CTAs instead: three tensor passes per byte
-            // make the lost L2 reuse cheap there (1024x8192x8192 measured 10%
-            // faster), while in TF32 it costs more than the idle CTAs.
+            // make the lost L2 reuse cheap there (measured faster: 10% on the
+            // pair plan of 1024x8192x8192, 14% on the swapped one-CTA plan of
+            // 128x32768x32768), while in TF32 it costs more than the idle CTAs.
             // (Only for fewer than two waves, where the idle share is large.)
-            const bool spread = hybrid || (pl.prec == fle::kPrec3xTF32 && S < 2 && pl.pair && T < 2 * G);
+            const bool spread = hybrid || (pl.prec == fle::kPrec3xTF32 && S < 2 && T < 2 * G);
             if (spread && T > G) {
                 pl.dp_tiles = static_cast<int>(T - R);
                 pl.grid = static_cast<int>(G);

@@ -230,3 +230,15 @@ def test_uneven_last_wave_spreads_only_in_3xtf32():
     load = [sum(int(r[4]) - int(r[3]) for r in rows) for rows in per]
     assert grid == 74 and _tiles(per) == 112
     assert sum(load) == 112 * 256 and max(load) - min(load) <= 1
+
+
+def test_swapped_3xtf32_spreads_its_uneven_last_wave():
+    # 128 x 32768 x 32768 in 3xTF32 runs the one-CTA swapped kernel: 256 weight
+    # tiles of 128 rows on 148 CTAs, one full wave and 108 tiles that cannot be
+    # split evenly (148 // 108 = 1).  Their k-blocks are spread over all 148
+    # CTAs, so every CTA does one whole tile and 747 or 748 k-blocks more.
+    d = fle.desc_for("swish_scale", "3xtf32")
+    grid, per = collect(128, 32768, 32768, d, 148)
+    load = [sum(int(r[4]) - int(r[3]) for r in rows) for rows in per]
+    assert grid == 148 and _tiles(per) == 256
+    assert sum(load) == 256 * 1024 and max(load) - min(load) <= 1
