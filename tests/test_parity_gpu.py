@@ -429,6 +429,65 @@ def test_swapped_pair_tiles(fle, M, problem):
     _assert_close(out.cpu().numpy(), _oracle(x, W, b, problem), "tf32", f"{M}x{K}x{N} {plan}")
 
 
+_PAIR_3X_SCRIPT = r"""
+import sys, numpy as np, torch
+import oracle
+import reduction_epilogue_b200 as fle
+from reduction_epilogue_b200 import synth
+lib = fle.load()
+bad = []
+for (M, K, N, problem) in [(128, 520, 75 * 256 - 93, "scale_hardtanh_gelu"), (45, 2080, 40 * 256, "swish_scale"),
+                           (100, 4096, 2000, "none"), (1, 1056, 19107, "swish_scale"),
+                           (64, 4096, 29100, "scale_hardtanh_gelu")]:
+    d = fle.desc_for(problem, "3xtf32")
+    plan = fle.plan_string(M, K, N, d)
+    if "pair=1 swap=1" not in plan:
+        bad.append(("not the swapped pair kernel", plan))
+        continue
+    x, W, b = synth.linear_inputs(M, K, N, seed=M + K, device="cuda")
+    outs = []
+    for mode in (1, 2, 0):  # FLE_FINISH_OWN, FLE_FINISH_LAST, FLE_FINISH_AUTO
+        lib.fle_test_set_finisher(mode)
+        out = fle.linear_epilogue(x, W, b, problem, "3xtf32")
+        torch.cuda.synchronize()
+        if fle.device_status() != 0:
+            bad.append(("status", M, K, N, mode, plan))
+        outs.append(out.cpu().numpy())
+    lib.fle_test_set_finisher(0)
+    if not all(np.array_equal(outs[0], o) for o in outs[1:]):
+        bad.append(("finisher branches differ", M, K, N, plan))
+    cols = np.arange(N) if N <= 20000 else np.unique(np.r_[0:256, N - 256:N, np.arange(0, N, 97)])
+    ref = oracle.forward_rows(x.cpu().numpy(), W.cpu().numpy()[cols], b.cpu().numpy()[cols],
+                              **oracle.PROBLEMS[problem]).astype(np.float64)
+    got = outs[0][:, cols].astype(np.float64)
+    err = np.abs(got - ref)
+    if not np.isfinite(got).all() or (err > 1e-4 + 1e-4 * np.abs(ref)).any():
+        bad.append(("oracle", M, K, N, problem, float(err.max()), plan))
+    print("PLAN", plan)
+print("BAD", bad)
+sys.exit(1 if bad else 0)
+"""
+
+
+def test_swapped_pair_tiles_3xtf32():
+    # The swapped pair kernel in 3xTF32 (FLE_PAIR=1 forces it for skinny M):
+    # ragged M, N and K, whole tiles, tiles split k-aligned over pairs and an
+    # uneven last wave spread over all pairs (64 x 4096 x 29100), both
+    # finisher branches bitwise equal, against the oracle at the 3xTF32
+    # tolerance (on a spread of output columns for the widest weight).
+    import os
+    import subprocess
+    import sys
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, FLE_PAIR="1", PYTHONPATH=root)
+    r = subprocess.run([sys.executable, "-c", _PAIR_3X_SCRIPT], cwd=root, env=env, capture_output=True, text=True,
+                       timeout=900)
+    assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-4000:]
+    assert r.stdout.count("PLAN tile=256x") == 5, r.stdout
+
+
 OPTION_SHAPES = [(7, 36, 33), (100, 1056, 520), (200, 64, 301), (300, 132, 1000), (128, 520, 19107)]
 
 
