@@ -267,6 +267,21 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             mma_commit_pair(bar_drain);
             volatile int never = 0;
             mbar_wait_bounded(bar_drain, 0, &never, kDrainTimeoutNs, kWhereDrain);
+            // Both CTAs' epilogues release each accumulator buffer with an
+            // arrival on this CTA's barrier, the peer's from the other SM.
+            // The last release of each buffer is never waited for by the loop
+            // above; wait for it here, so that no arrival from the peer is
+            // still on its way to this CTA's shared memory when it exits (it
+            // would land in whichever CTA runs on this SM next).
+            for (int i = 0; ok && i < C::kNumAcc; ++i) {
+                if (!mbar_wait_bounded(bar_acce(buf), acc_phase ^ 1u, abort_flag, p.timeout_ns, kWhereDrain,
+                                       peer_abort))
+                    break;
+                if (++buf == C::kNumAcc) {
+                    buf = 0;
+                    acc_phase ^= 1u;
+                }
+            }
         }
         __syncwarp();
     } else if (warp < 4) {
@@ -549,6 +564,9 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         mbar_arrive_cluster(mapa_shared(bar_exit, rank ^ 1u));
         volatile int never = 0;
         mbar_wait_bounded(bar_exit, 0, &never, p.timeout_ns + 2 * kDrainTimeoutNs, kWhereDrain);
+        // the wait acquires at CTA scope; the other CTA released at cluster
+        // scope: order this CTA's teardown after everything it did before
+        fence_acq_rel_cluster();
     }
     __syncwarp();
     __syncthreads();

@@ -198,6 +198,11 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 
 // Orders this thread's generic-proxy shared-memory writes before later
 // async-proxy reads of the same bytes (tcgen05.mma operands).
+// Acquire-release fence at cluster scope: after observing another CTA's
+// release (an arrival on a barrier here), this thread's later accesses are
+// ordered after everything that CTA ordered before its release.
+__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
