@@ -62,7 +62,10 @@ struct PairCfg {
                                     : (kTmemAll <= 128) ? 128 : (kTmemAll <= 256) ? 256 : 512;
     // full, split, empty per stage; accf, acce per buffer; drain; exit
     static constexpr int kNumBars = 3 * kStages + 4 + 2;
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kEpiStageBytes + kNumBars * 8 + 32;
+    // (the checking build keeps its stage and accumulator tags after the 32
+    // bytes of TMEM address and flags)
+    static constexpr int kSmemBytes =
+        1024 + kStages * kStageBytes + kEpiStageBytes + kNumBars * 8 + 32 + (kCheckBarriers ? 64 : 0);
     static_assert(kStages >= 2, "need at least two stages");
     static_assert(KPS == 1 || KPS == 2, "one or two k-blocks per stage");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 512, "pair tile N: 32..512, whole 32-column chunks");
@@ -96,6 +99,12 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     // two slots used in turn (see fle_gemm_kernel)
     volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+    // checking build: the work tag of each stage (per CTA) and of each
+    // accumulator buffer (in the leader)
+    volatile uint32_t* stage_tag = reinterpret_cast<volatile uint32_t*>(tmem_slot + 8);
+    volatile uint32_t* acc_tag = stage_tag + 12;
+    (void)stage_tag;
+    (void)acc_tag;
 
     auto bar_full = [&](int s) { return smem_u32(bars + s); };
     auto bar_split = [&](int s) { return smem_u32(bars + S + s); };
@@ -165,6 +174,13 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                         ok = false;
                         break;
                     }
+                    if constexpr (kCheckBarriers) {
+                        // the full barrier in use: each CTA's own (3xTF32), the leader's (TF32)
+                        if ((k3x || rank == 0) && mbar_test_wait(bar_full(stage), phase))
+                            record_error(kErrProtocol, kWhereProdEmpty);
+                        stage_tag[stage] = work_tag(u.t, kb);
+                        fence_acq_rel_cluster();
+                    }
                     if constexpr (k3x) {
                         // own barrier: this CTA's split warps wait for these bytes
                         mbar_arrive_expect_tx(bar_full(stage), n * C::kKbBytes);
@@ -220,6 +236,10 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                         break;
                     }
                     tc_fence_after_sync();
+                    if constexpr (kCheckBarriers) {
+                        acc_tag[buf] = work_tag(u.t, kc);
+                        fence_acq_rel_cluster();
+                    }
                     const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * C::kAccCols);
                     for (int kb = kc; kb < kce; kb += KPS) {
                         const int n = (kce - kb < KPS) ? kce - kb : KPS;  // k-blocks in this stage
@@ -229,6 +249,13 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                             break;
                         }
                         tc_fence_after_sync();
+                        if constexpr (kCheckBarriers) {
+                            // this CTA's stage and the peer's hold the same work
+                            const uint32_t want = work_tag(u.t, kb);
+                            check_tag(stage_tag[stage], want, kWhereMmaFull);
+                            check_tag(ld_cluster_u32(mapa_shared(smem_u32(const_cast<uint32_t*>(stage_tag + stage)), 1)),
+                                      want, kWhereMmaFull);
+                        }
                         auto desc = [](uint32_t a) { return smem_desc_sw128(a); };
                         for (int j = 0; j < n; ++j) {
                             const uint64_t a_hi = desc(sA(stage) + j * C::kABytes);
@@ -301,6 +328,10 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                         got = mbar_wait_bounded(bar_full(stage), phase, abort_flag, p.timeout_ns, kWhereConvFull, peer_abort);
                     got = __shfl_sync(0xffffffffu, got, 0);
                     if (!got) { ok = false; break; }
+                    if constexpr (kCheckBarriers) {
+                        if (lane == 0) check_tag(stage_tag[stage], work_tag(u.t, kb), kWhereConvFull);
+                        __syncwarp();
+                    }
                     const float4* x4 = reinterpret_cast<const float4*>(smem + stage * C::kStageBytes);
                     float4* lo4 = reinterpret_cast<float4*>(smem + stage * C::kStageBytes + C::kLoadBytes);
                     constexpr int kVec = C::kLoadBytes / 16;
@@ -351,10 +382,18 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             Unit uh = u;
             uh.ta = 2 * u.ta + static_cast<int>(rank);
             eo.row0 = static_cast<int64_t>(uh.ta) * kBM + q * 32;
-            auto wait_acc = [&]() -> bool {
+            auto wait_acc = [&](int kc) -> bool {
                 int got = 0;
-                if (lane == 0)
+                if (lane == 0) {
                     got = mbar_wait_bounded(bar_accf(buf), acc_phase, abort_flag, p.timeout_ns, kWhereEpiAccFull, peer_abort);
+                    if constexpr (kCheckBarriers) {
+                        // the leader's MMA tagged the buffer it filled
+                        if (got)
+                            check_tag(ld_cluster_u32(mapa_shared(smem_u32(const_cast<uint32_t*>(acc_tag + buf)), 0)),
+                                      work_tag(u.t, kc), kWhereEpiAccFull);
+                    }
+                }
+                (void)kc;
                 got = __shfl_sync(0xffffffffu, got, 0);
                 if (got) tc_fence_after_sync();
                 return got != 0;
@@ -378,7 +417,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
 #pragma unroll
                 for (int j = 0; j < kHalf * 32; ++j) accr[j] = 0.0f;
                 for (int kc = u.kb0; kc < u.kb1; kc += kChunkKb) {
-                    if (!wait_acc()) { ok = false; break; }
+                    if (!wait_acc(kc)) { ok = false; break; }
                     const uint32_t tr = t_row();
 #pragma unroll
                     for (int lc = 0; lc < kHalf; ++lc) {
@@ -395,7 +434,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 }
                 if (!ok) break;
             } else {
-                if (!wait_acc()) break;
+                if (!wait_acc(u.kb0)) break;
                 t_acc = t_row();
             }
 

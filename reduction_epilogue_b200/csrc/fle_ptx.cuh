@@ -92,8 +92,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // ----------------------------------------------------------------------------
-// Barrier-protocol checks (a build with -DFLE_CHECK_BARRIERS; the one-CTA
-// kernel).  The producer of each ring stage and of each TMEM accumulator
+// Barrier-protocol checks (a build with -DFLE_CHECK_BARRIERS; both
+// kernels).  The producer of each ring stage and of each TMEM accumulator
 // writes a tag naming the work it holds (tile, first k-block) next to it;
 // every consumer, after its barrier wait, compares that tag with the work its
 // own walk of the schedule expects, and records status 10 (FLE_ERR_PROTOCOL)
@@ -130,6 +130,13 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
         : "r"(bar), "r"(parity)
         : "memory");
     return ok != 0;
+}
+
+// A 32-bit word in shared memory of a CTA of this cluster (address from mapa).
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t remote_addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(remote_addr) : "memory");
+    return v;
 }
 
 // Stores a 32-bit word into shared memory of a CTA of this cluster (address

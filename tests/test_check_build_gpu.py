@@ -1,19 +1,21 @@
 """The barrier-checking build on the GPU.
 
-libfle_check.so is the library compiled with -DFLE_CHECK_BARRIERS.  In its
-one-CTA kernel every ring stage and every TMEM accumulator carries a tag
-naming the work (tile, first k-block) its producer put there, and each
-consumer compares it, after its barrier wait, with the work its own walk of
-the schedule expects; a mismatch, or a producer re-arming a stage whose
+libfle_check.so is the library compiled with -DFLE_CHECK_BARRIERS.  In both
+kernels every ring stage and every TMEM accumulator carries a tag naming the
+work (tile, first k-block) its producer put there, and each consumer compares
+it, after its barrier wait, with the work its own walk of the schedule
+expects; in the CTA-pair kernel the leader's MMA also reads the peer CTA's
+stage tags, and the peer's epilogue the leader's accumulator tags, through
+distributed shared memory.  A mismatch, or a producer re-arming a stage whose
 phase already completed, records FLE_ERR_PROTOCOL in the device status word.
 These checks stand in for a race detector (compute-sanitizer is not
-available here).  The CTA-pair kernel is the same in both libraries.  The
-one-CTA kernel runs for every shape here under FLE_PAIR=0 (direct and
-swapped layouts), and under an even stream-K spread (FLE_SCHED=sk: short
-units, CTAs holding two shared tiles); the default plans mix both kernels.
-Each variant runs in a fresh process (the planner overrides are read once
-per process) and must end with a clean status and results that match the
-oracle.
+available here).  Variants: the default plans (both kernels), the one-CTA
+kernel alone (FLE_PAIR=0) and under an even stream-K spread (FLE_SCHED=sk:
+short units, CTAs holding two shared tiles), the pair kernel under the same
+spread, and 256-wide pair tiles of one k-block per stage (FLE_PAIR_BN=256
+FLE_KPS=1).  Each variant runs in a fresh process (the planner overrides are
+read once per process) and must end with a clean status and results that
+match the oracle.
 """
 import os
 import subprocess
@@ -59,9 +61,11 @@ print("BAD", bad)
 sys.exit(1 if bad else 0)
 """
 
-# planner overrides: the default plans, one-CTA tiles only, and an even
-# stream-K spread on one-CTA tiles
-VARIANTS = [{}, {"FLE_PAIR": "0"}, {"FLE_PAIR": "0", "FLE_SCHED": "sk"}]
+# planner overrides: the default plans, one-CTA tiles only, an even stream-K
+# spread on one-CTA tiles and on pair tiles, and 256-wide pair tiles of one
+# k-block per stage
+VARIANTS = [{}, {"FLE_PAIR": "0"}, {"FLE_PAIR": "0", "FLE_SCHED": "sk"}, {"FLE_SCHED": "sk"},
+            {"FLE_PAIR_BN": "256", "FLE_KPS": "1"}]
 
 
 @pytest.fixture(scope="module")
