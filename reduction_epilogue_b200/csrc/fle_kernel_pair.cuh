@@ -1,13 +1,15 @@
 // fle_kernel_pair.cuh -- the fused Linear + epilogue kernel on CTA pairs.
 //
-// Two CTAs of a cluster, on two SMs, compute one 256 x 256 output tile with
-// tcgen05.mma.cta_group::2: each CTA loads its own 128 rows of A (x) and its
-// own 128 rows of B (W) into its shared memory, and the pair's MMA reads A and
+// Two CTAs of a cluster, on two SMs, compute one output tile of 256 A rows
+// with tcgen05.mma.cta_group::2: each CTA loads its own 128 rows of A and its
+// half of the B rows into its shared memory, and the pair's MMA reads A and
 // B from both.  Per SM this halves the B operand traffic through shared memory
-// compared with a 128 x 256 single-CTA tile, at the same MMA work per SM.
-// The accumulator rows are split across the two SMs' TMEM (rows 0-127 in the
-// even CTA, 128-255 in the odd one), so each CTA runs the epilogue of its own
-// 128 rows.
+// compared with a single-CTA tile, at the same MMA work per SM.  The
+// accumulator rows are split across the two SMs' TMEM (rows 0-127 in the even
+// CTA, 128-255 in the odd one), so each CTA runs the epilogue of its own 128
+// rows.  Tile widths (B rows): 256 or 224 (direct order), 512 (two 256-wide
+// MMAs per k-step sharing the A tile, single-pass TF32), and 32, 64 or 128
+// in the swapped order (A = W, B = x) of the skinny shapes.
 //
 // Roles are those of fle_gemm_kernel.  Only the even ("leader") CTA's MMA
 // thread issues MMAs; the leader's commits are multicast to both CTAs' empty
@@ -21,6 +23,10 @@
 //           barrier, which the MMA waits on.  The three products of each
 //           k-step accumulate in 128-deep slices of K, summed in registers
 //           (the tensor core's own accumulation rounds toward zero).
+// Every signal one CTA sends the other is waited for before the receiver
+// exits (the last accumulator releases by the leader's MMA thread, the rest
+// by the roles that consume them, then a bounded two-way handshake), so no
+// arrival can reach the shared memory of the next CTA on that SM.
 #pragma once
 
 #include "fle_kernel.cuh"
