@@ -149,7 +149,7 @@ int check_shape(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d) {
 
 struct Plan {
     bool swap = false;
-    bool pair = false;         // 256x256 tiles on CTA pairs (cta_group::2)
+    bool pair = false;         // tiles of 256 A rows on CTA pairs (cta_group::2)
     int kps = 1;               // k-blocks per ring stage
     int bk = 32;               // k-block width in fp32
     int bn = 256;
