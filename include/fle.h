@@ -200,12 +200,15 @@ int fle_plan_string(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* de
 
 /* Introspection of the launch plan; needs no GPU.  Lists the work units that
  * CTA `cta` of the plan for (M,K,N,desc) on a device with num_sms SMs would
- * run, in order, as 10 int32 per unit:
+ * run, in order, as 12 int32 per unit:
  *   tile, tile_a, tile_b, kb_begin, kb_end, partial, slot,
- *   first_contributor, last_contributor, slot_by_rule
- * (the last four are -1 for a tile this CTA computes whole; for a shared
- * tile they are its workspace slot, the range of CTAs that share it, and the
- * slot the finishing CTA will read for this CTA).  Writes at most max_units
+ *   first_contributor, last_contributor, slot_by_rule, b_begin, b_width
+ * (slot .. slot_by_rule are -1 for a tile this CTA computes whole; for a
+ * shared tile they are its workspace slot, the range of CTAs that share it,
+ * and the slot the finishing CTA will read for this CTA.  b_begin and
+ * b_width are the tile's first operand-B row (output column, or output row
+ * in the swapped order) and its number of B rows; tile_b is -1 in a plan of
+ * mixed tile widths, whose tiles are not on one grid).  Writes at most max_units
  * rows to units (host memory); *n_units receives the total count and *grid
  * (if not NULL) the plan's grid size.  Returns FLE_OK or an argument error. */
 int fle_plan_units(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* desc, int num_sms,

@@ -204,7 +204,7 @@ def plan_units(M: int, K: int, N: int, desc: EpilogueDesc, num_sms: int, cta: in
     st = lib.fle_plan_units(M, K, N, ctypes.byref(desc), num_sms, cta, None, 0, ctypes.byref(n), ctypes.byref(g))
     if st != FLE_OK:
         raise FleError(st, "fle_plan_units")
-    rows = np.zeros((max(n.value, 1), 10), dtype=np.int32)
+    rows = np.zeros((max(n.value, 1), 12), dtype=np.int32)
     st = lib.fle_plan_units(M, K, N, ctypes.byref(desc), num_sms, cta, rows.ctypes.data, n.value,
                             ctypes.byref(n), ctypes.byref(g))
     if st != FLE_OK:

@@ -11,6 +11,7 @@
 #include <atomic>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "fle.h"
 #include "fle_testing.h"
@@ -165,6 +166,11 @@ struct Plan {
     int grid = 0;
     size_t partial_bytes = 0;  // workspace: 2 partial tiles per CTA ...
     size_t ws_bytes = 0;       // ... then one arrival counter per stream-K tile
+    // mixed widths (512-wide pair kernel): mix_wide 512-wide tiles, then
+    // mix_narrow 384-wide ones; per panel, mix_a[r] and mix_b[r] of them
+    int mix_wide = 0, mix_narrow = 0;
+    unsigned char mix_a[fle::kMaxMixPanels] = {};
+    unsigned char mix_b[fle::kMaxMixPanels] = {};
 };
 
 // Ring depth of the single-CTA kernel (mirrors Cfg::kStages).
@@ -219,6 +225,60 @@ int pair_bn_override() {
         return (n == fle::kPairBN || n == fle::kPairBNNarrow || n == fle::kPairBNWide) ? n : 0;
     }();
     return v;
+}
+
+// FLE_MIX=0 keeps the 512-wide plans on a uniform grid (comparisons).
+bool mix_disabled() {
+    static bool off = [] {
+        const char* e = std::getenv("FLE_MIX");
+        return e && e[0] == '0';
+    }();
+    return off;
+}
+
+// Mixed widths for a 512-wide plan of more than one wave on G pairs: each
+// 256-row panel r is cut into a[r] tiles 512 wide, then b[r] = ceil((N -
+// 512 a[r]) / 384) tiles 384 wide, with at most G tiles of each width, so
+// that every pair runs at most one of each.  The cut takes one or two values
+// of a[r] (n1 panels at a1, the rest at a2): the most 512-wide tiles, then
+// the most even split, so that the tiles of each wave share operand rows
+// across panels.  Returns false when there is no such cut.
+bool mixed_cut(int64_t panels, int64_t N, int64_t G, unsigned char* a_out, unsigned char* b_out, int* n_wide,
+               int* n_narrow) {
+    if (panels < 1 || panels > fle::kMaxMixPanels || G < 1) return false;
+    const int64_t A = (N + fle::kMixWide - 1) / fle::kMixWide;
+    if (A > 255) return false;
+    auto b_of = [&](int64_t a) {
+        const int64_t rest = N - fle::kMixWide * a;
+        return rest > 0 ? (rest + fle::kMixNarrow - 1) / fle::kMixNarrow : int64_t(0);
+    };
+    int64_t best_wide = -1, best_spread = 0, best_a1 = 0, best_a2 = 0, best_n1 = 0;
+    for (int64_t a1 = 0; a1 <= A; ++a1)
+        for (int64_t a2 = a1; a2 <= A; ++a2)
+            for (int64_t n1 = (a1 == a2 ? panels : 1); n1 <= panels; ++n1) {
+                const int64_t wide = n1 * a1 + (panels - n1) * a2;
+                const int64_t narrow = n1 * b_of(a1) + (panels - n1) * b_of(a2);
+                if (wide > G || narrow > G || b_of(a1) > 255) continue;
+                const int64_t spread = a2 - a1;
+                if (wide > best_wide || (wide == best_wide && spread < best_spread)) {
+                    best_wide = wide;
+                    best_spread = spread;
+                    best_a1 = a1;
+                    best_a2 = a2;
+                    best_n1 = n1;
+                }
+            }
+    if (best_wide < 0) return false;
+    int narrow = 0;
+    for (int64_t r = 0; r < panels; ++r) {
+        const int64_t a = r < best_n1 ? best_a1 : best_a2;
+        a_out[r] = static_cast<unsigned char>(a);
+        b_out[r] = static_cast<unsigned char>(b_of(a));
+        narrow += b_out[r];
+    }
+    *n_wide = static_cast<int>(best_wide);
+    *n_narrow = narrow;
+    return true;
 }
 
 // FLE_PAIR=0 keeps every plan on one-CTA tiles; FLE_PAIR=1 puts every
@@ -306,6 +366,21 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
             if (Tw % G != 0 && ww != std::floor(ww)) ww += 0.25;  // split last wave of wide partials
             const double c512 = 0.86 * fle::kPairBNWide * ww;
             if (c512 < 0.985 * std::min(c256, c224)) pl.bn = fle::kPairBNWide;
+            // Mixed widths: a plan of more than one wave of 512-wide tiles
+            // whose last wave is short (2048 x 8192 x 8192: 128 tiles on 74
+            // pairs, the second wave 54) can run one wave of 512-wide tiles
+            // and one of 384-wide ones (74 + 73 tiles): each pair then does
+            // 896 columns instead of 1024.  A 384-wide tile is a 256-wide and
+            // a 128-wide MMA sharing the A tile; the narrow MMA reads the
+            // whole A tile for half the columns, so a column costs 1.25x a
+            // 512-wide one (measured on 2048 x 8192 x 8192: 178 against
+            // 190 us per wave, and 368 against 380 us for the whole plan).
+            if (Tw > G && pair_bn_override() == 0 && !mix_disabled()) {
+                const double cmix = 0.86 * (fle::kMixWide + 1.25 * fle::kMixNarrow);
+                if (cmix < 0.985 * std::min(std::min(c256, c224), c512) &&
+                    mixed_cut(ta, N, G, pl.mix_a, pl.mix_b, &pl.mix_wide, &pl.mix_narrow))
+                    pl.bn = fle::kPairBNWide;
+            }
         }
         if (pair_bn_override() != 0) pl.bn = pair_bn_override();
         if (pl.bn > 256 && pl.prec != fle::kPrecTF32) pl.bn = fle::kPairBN;  // wide tiles: TF32 only
@@ -316,7 +391,7 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
     const int64_t Nb = pl.swap ? M : N;
     pl.tiles_a = static_cast<int>((Ma + tile_m - 1) / tile_m);
     pl.tiles_b = static_cast<int>((Nb + pl.bn - 1) / pl.bn);
-    pl.tiles = pl.tiles_a * pl.tiles_b;
+    pl.tiles = pl.mix_wide > 0 ? pl.mix_wide + pl.mix_narrow : pl.tiles_a * pl.tiles_b;
     pl.bk = fle::kBK;
     pl.num_kb = static_cast<int>((K + pl.bk - 1) / pl.bk);
     // Two k-blocks per ring stage (TF32): measured faster on the swapped
@@ -342,6 +417,7 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
     pl.dp_tiles = static_cast<int>(T);
     pl.grid = static_cast<int>(T < G ? T : G);
     pl.sk_grid = 0;
+    if (pl.mix_wide > 0) return pl;  // at most two tiles per pair, all whole
     // Splitting K costs a partial-tile round trip and a wait at the end of the
     // tile (a few microseconds); it is taken only for tiles of at least four
     // minimum-size parts (measured: at K = 1024 the whole tiles are faster).
@@ -435,8 +511,8 @@ cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
 }
 
 template <int PREC, int KPS, int BN = fle::kPairBN, bool SWAP = false>
-cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to, const KParams& p,
-                             int pairs, bool after_prep, cudaStream_t st) {
+cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb2,
+                             const CUtensorMap& to, const KParams& p, int pairs, bool after_prep, cudaStream_t st) {
     using C = fle::PairCfg<PREC, KPS, BN, SWAP>;
     auto kern = fle::fle_gemm_pair_kernel<PREC, KPS, BN, SWAP>;
     static std::atomic<bool> attr_set[kMaxDevices] = {};
@@ -461,35 +537,36 @@ cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = after_prep ? 2 : 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, to, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tb2, to, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
-cudaError_t dispatch(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
-                     const KParams& p, bool after_prep, cudaStream_t st) {
+// tb2: the 64-row boxes of B for the 384-wide tiles of a mixed plan (else tb).
+cudaError_t dispatch(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb2,
+                     const CUtensorMap& to, const KParams& p, bool after_prep, cudaStream_t st) {
     using namespace fle;
     const bool tf32 = pl.prec == kPrecTF32;
     const bool two = pl.kps == 2;  // TF32 only
     if (pl.pair && !pl.swap && pl.bn == kPairBNWide)
-        return launch_gemm_pair<kPrecTF32, 1, kPairBNWide>(ta, tb, to, p, pl.grid, after_prep, st);
+        return launch_gemm_pair<kPrecTF32, 1, kPairBNWide>(ta, tb, tb2, to, p, pl.grid, after_prep, st);
     if (pl.pair && !pl.swap && pl.bn == kPairBNNarrow) {
-        if (!tf32) return launch_gemm_pair<kPrec3xTF32, 1, kPairBNNarrow>(ta, tb, to, p, pl.grid, after_prep, st);
-        return two ? launch_gemm_pair<kPrecTF32, 2, kPairBNNarrow>(ta, tb, to, p, pl.grid, after_prep, st)
-                   : launch_gemm_pair<kPrecTF32, 1, kPairBNNarrow>(ta, tb, to, p, pl.grid, after_prep, st);
+        if (!tf32) return launch_gemm_pair<kPrec3xTF32, 1, kPairBNNarrow>(ta, tb, tb2, to, p, pl.grid, after_prep, st);
+        return two ? launch_gemm_pair<kPrecTF32, 2, kPairBNNarrow>(ta, tb, tb2, to, p, pl.grid, after_prep, st)
+                   : launch_gemm_pair<kPrecTF32, 1, kPairBNNarrow>(ta, tb, tb2, to, p, pl.grid, after_prep, st);
     }
     if (pl.pair && !pl.swap) {
-        if (!tf32) return launch_gemm_pair<kPrec3xTF32, 1>(ta, tb, to, p, pl.grid, after_prep, st);
-        return two ? launch_gemm_pair<kPrecTF32, 2>(ta, tb, to, p, pl.grid, after_prep, st)
-                   : launch_gemm_pair<kPrecTF32, 1>(ta, tb, to, p, pl.grid, after_prep, st);
+        if (!tf32) return launch_gemm_pair<kPrec3xTF32, 1>(ta, tb, tb2, to, p, pl.grid, after_prep, st);
+        return two ? launch_gemm_pair<kPrecTF32, 2>(ta, tb, tb2, to, p, pl.grid, after_prep, st)
+                   : launch_gemm_pair<kPrecTF32, 1>(ta, tb, tb2, to, p, pl.grid, after_prep, st);
     }
     if (pl.pair) {
         switch (pl.bn) {
 #define FLE_PAIR_SWAP_CASE(bn)                                                                             \
     case bn:                                                                                               \
-        if (!tf32) return launch_gemm_pair<kPrec3xTF32, 1, bn, true>(ta, tb, to, p, pl.grid, after_prep, st); \
-        return two ? launch_gemm_pair<kPrecTF32, 2, bn, true>(ta, tb, to, p, pl.grid, after_prep, st)      \
-                   : launch_gemm_pair<kPrecTF32, 1, bn, true>(ta, tb, to, p, pl.grid, after_prep, st);
+        if (!tf32) return launch_gemm_pair<kPrec3xTF32, 1, bn, true>(ta, tb, tb2, to, p, pl.grid, after_prep, st); \
+        return two ? launch_gemm_pair<kPrecTF32, 2, bn, true>(ta, tb, tb2, to, p, pl.grid, after_prep, st)      \
+                   : launch_gemm_pair<kPrecTF32, 1, bn, true>(ta, tb, tb2, to, p, pl.grid, after_prep, st);
             FLE_PAIR_SWAP_CASE(32)
             FLE_PAIR_SWAP_CASE(64)
             FLE_PAIR_SWAP_CASE(128)
@@ -559,6 +636,12 @@ int plan_to_string(const Plan& pl, char* buf, size_t n) {
                   pl.prec == fle::kPrecTF32 ? "tf32" : "3xtf32", pl.stages, pl.kps,
                   pl.tiles_a, pl.tiles_b, pl.num_kb, pl.dp_tiles, pl.sk_tiles, (long long)pl.sk_iters, pl.sk_grid,
                   pl.sk_slots, pl.grid, pl.ws_bytes);
+    if (pl.mix_wide > 0) {
+        const size_t used = std::strlen(buf);
+        if (used + 1 < n)
+            std::snprintf(buf + used, n - used, " mix=%dx%d+%dx%d", pl.mix_wide, fle::kMixWide, pl.mix_narrow,
+                          fle::kMixNarrow);
+    }
     return FLE_OK;
 }
 
@@ -681,12 +764,16 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
     p.sk_iters = pl.sk_iters;
     p.sk_grid = pl.sk_grid;
     p.sk_slots = pl.sk_slots;
+    p.tile_n = pl.bn;
+    p.mix_wide = pl.mix_wide;
+    std::memcpy(p.mix_a, pl.mix_a, sizeof p.mix_a);
+    std::memcpy(p.mix_b, pl.mix_b, sizeof p.mix_b);
     if (pl.sk_tiles > 0) {
         p.ws = static_cast<float*>(workspace);
         p.counters = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + pl.partial_bytes);
     }
 
-    CUtensorMap ta, tb, to;
+    CUtensorMap ta, tb, tb2, to;
     std::memset(&to, 0, sizeof to);
     // Elementwise kinds (direct or swapped layout) store through TMA when the
     // output rows are 16-byte multiples and the base is 16-byte aligned.
@@ -703,6 +790,12 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
     // tile (each CTA loads its 128 rows of both 256-wide sub-tiles)
     st = encode_operand(&tb, B, p.Nb, K, pl.pair ? (pl.bn > 256 ? 128 : pl.bn / 2) : pl.bn);
     if (st != FLE_OK) return st;
+    // a mixed plan's 384-wide tiles: 64 rows per CTA of their 128-wide sub-tile
+    tb2 = tb;
+    if (pl.mix_wide > 0) {
+        st = encode_operand(&tb2, B, p.Nb, K, (fle::kMixNarrow - 256) / 2);
+        if (st != FLE_OK) return st;
+    }
 
     if (log_enabled()) {
         char line[256];
@@ -720,7 +813,7 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
             pool ? out : nullptr, pool ? M : 0, p.counters, n_counters);
         if (cudaGetLastError() != cudaSuccess) return FLE_ERR_CUDA;
     }
-    if (dispatch(pl, ta, tb, to, p, prep, s) != cudaSuccess) return FLE_ERR_CUDA;
+    if (dispatch(pl, ta, tb, tb2, to, p, prep, s) != cudaSuccess) return FLE_ERR_CUDA;
     if (sync_check_enabled()) return fle_device_status(stream);
     return FLE_OK;
 }
@@ -747,14 +840,20 @@ int fle_plan_units(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, 
     p.sk_iters = pl.sk_iters;
     p.sk_grid = pl.sk_grid;
     p.sk_slots = pl.sk_slots;
+    p.tile_n = pl.bn;
+    p.mix_wide = pl.mix_wide;
+    std::memcpy(p.mix_a, pl.mix_a, sizeof p.mix_a);
+    std::memcpy(p.mix_b, pl.mix_b, sizeof p.mix_b);
     fle::Sched sc;
     sc.init(p, cta, pl.grid);
     fle::Unit u;
     int n = 0;
     while (sc.next(p, u)) {
         if (n < max_units) {
-            int32_t* row = units + static_cast<size_t>(n) * 10;
+            int32_t* row = units + static_cast<size_t>(n) * 12;
             row[0] = u.t; row[1] = u.ta; row[2] = u.tb; row[3] = u.kb0; row[4] = u.kb1;
+            row[10] = static_cast<int32_t>(u.col0);
+            row[11] = u.w;
             row[5] = u.partial; row[6] = u.partial ? u.slot : -1;
             if (u.partial) {
                 row[7] = fle::sk_cta_of(static_cast<int64_t>(u.sk_tile) * p.num_kb, p.sk_iters, pl.sk_grid);

@@ -36,6 +36,10 @@ namespace fle {
 
 constexpr int kBM = 128;           // MMA M: rows of operand A per tile
 constexpr int kBK = 32;            // fp32 per k-block = one 128-byte swizzled row
+// Mixed-width plans (see KParams): tile widths and the most 256-row panels
+constexpr int kMixWide = 512;
+constexpr int kMixNarrow = 384;
+constexpr int kMaxMixPanels = 16;
 constexpr int kUmmaK = 8;          // K of one tcgen05.mma kind::tf32
 constexpr int kThreads = 384;
 constexpr int kEpiWarps = 8;                 // warps 4..11
@@ -80,11 +84,21 @@ struct KParams {
     int vec_bias;           // bias 16-byte aligned
     int tma_out;            // direct layout: write out through TMA tile stores
     uint64_t timeout_ns;
+    int tile_n;             // B rows per tile (the kernel's tile width)
+    // Mixed-width plans of the 512-wide pair kernel (data-parallel only):
+    // each 256-row panel r holds mix_a[r] tiles 512 wide from column 0, then
+    // mix_b[r] tiles 384 wide.  Units [0, mix_wide) are the 512-wide tiles,
+    // panel by panel, the rest the 384-wide ones.  0: a uniform grid of tiles.
+    int mix_wide;
+    unsigned char mix_a[kMaxMixPanels];
+    unsigned char mix_b[kMaxMixPanels];
 };
 
 // One unit of work: tile t over k-blocks [kb0, kb1).
 struct Unit {
-    int t, ta, tb;
+    int t, ta, tb;          // tile; its index along A rows and along B rows (-1: mixed plan)
+    int64_t col0;           // first B row of the tile
+    int w;                  // B rows of the tile
     int kb0, kb1;
     int partial;            // the tile's k-range is shared with other CTAs
     int sk_tile;            // index among the stream-K tiles
@@ -133,8 +147,27 @@ struct Sched {
         } else {
             return false;
         }
-        u.ta = u.t % p.tiles_a;
-        u.tb = u.t / p.tiles_a;
+        if (p.mix_wide > 0) {
+            // mixed widths: walk the panels to the unit's tile
+            const bool wide = u.t < p.mix_wide;
+            int i = wide ? u.t : u.t - p.mix_wide;
+            int r = 0;
+            for (; r + 1 < p.tiles_a; ++r) {
+                const int n = wide ? p.mix_a[r] : p.mix_b[r];
+                if (i < n) break;
+                i -= n;
+            }
+            u.ta = r;
+            u.tb = -1;
+            u.w = wide ? kMixWide : kMixNarrow;
+            u.col0 = wide ? static_cast<int64_t>(kMixWide) * i
+                          : static_cast<int64_t>(kMixWide) * p.mix_a[r] + static_cast<int64_t>(kMixNarrow) * i;
+        } else {
+            u.ta = u.t % p.tiles_a;
+            u.tb = u.t / p.tiles_a;
+            u.w = p.tile_n;
+            u.col0 = static_cast<int64_t>(u.tb) * p.tile_n;
+        }
         return true;
     }
 };
@@ -455,7 +488,7 @@ __device__ __forceinline__ void epi_chunk(const KParams& p, const Unit& u, int r
                                           float& best, const EpiOut& eo) {
     if constexpr (!SWAP) {
         const int64_t m = static_cast<int64_t>(u.ta) * kBM + r;
-        const int64_t n0 = static_cast<int64_t>(u.tb) * BN + c * 32;
+        const int64_t n0 = u.col0 + c * 32;
         switch (p.kind) {
             case kEpiHardtanhGelu: epi_store_direct<kEpiHardtanhGelu>(p, eo, m, n0, v); break;
             case kEpiSwish: epi_store_direct<kEpiSwish>(p, eo, m, n0, v); break;
@@ -464,7 +497,7 @@ __device__ __forceinline__ void epi_chunk(const KParams& p, const Unit& u, int r
         }
     } else {
         const int64_t n = static_cast<int64_t>(u.ta) * kBM + r;
-        const int64_t m0 = static_cast<int64_t>(u.tb) * BN + c * 32;
+        const int64_t m0 = u.col0 + c * 32;
         switch (p.kind) {
             case kEpiHardtanhGelu: epi_store_swapped<kEpiHardtanhGelu>(p, eo, n, m0, v); break;
             case kEpiSwish: epi_store_swapped<kEpiSwish>(p, eo, n, m0, v); break;

@@ -9,7 +9,10 @@
 // CTA, 128-255 in the odd one), so each CTA runs the epilogue of its own 128
 // rows.  Tile widths (B rows): 256 or 224 (direct order), 512 (two 256-wide
 // MMAs per k-step sharing the A tile, single-pass TF32), and 32, 64 or 128
-// in the swapped order (A = W, B = x) of the skinny shapes.
+// in the swapped order (A = W, B = x) of the skinny shapes.  The 512-wide
+// kernel also runs mixed-width plans (KParams::mix_wide): 384-wide tiles are
+// a 256-wide and a 128-wide MMA sharing the A tile, whose 64 B rows per CTA
+// come through a second tensor map (tmB2, 64-row boxes).
 //
 // Roles are those of fle_gemm_kernel.  Only the even ("leader") CTA's MMA
 // thread issues MMAs; the leader's commits are multicast to both CTAs' empty
@@ -87,11 +90,19 @@ struct PairCfg {
 template <int PREC, int KPS, int BN, bool SWAP>
 __global__ void __launch_bounds__(kThreads, 1)
 fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmOut, const KParams p) {
+                     const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmOut,
+                     const KParams p) {
     using C = PairCfg<PREC, KPS, BN, SWAP>;
     constexpr bool k3x = (PREC == kPrec3xTF32);
     constexpr int S = C::kStages;
     constexpr uint32_t kIdesc = idesc_tf32(kPairBM, C::kSubN);
+    // 512-wide kernel: a 384-wide unit's second MMA is 128 wide (64 B rows
+    // per CTA, the first half of the sub-tile's slot)
+    constexpr bool kWide = BN > 256;
+    constexpr int kNarrowSubN = kMixNarrow - 256;
+    constexpr uint32_t kIdescNarrow = idesc_tf32(kPairBM, kNarrowSubN);
+    static_assert(!kWide || (BN == kMixWide && C::kNSub == 2 && C::kSubN == 256),
+                  "mixed plans: 512-wide tiles of two 256-wide sub-tiles");
     constexpr int kBKW = C::kBKW;
     constexpr int kChunkKb = k3x ? 128 / kBKW : (1 << 30);  // k-blocks per TMEM accumulation chain
     static_assert(kChunkKb % KPS == 0, "accumulation chains hold whole stages");
@@ -148,6 +159,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         fence_barrier_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if (kWide && p.mix_wide > 0) tma_prefetch_desc(&tmB2);
     }
     if (warp == 1) {
         tmem_alloc_pair(smem_u32(tmem_slot), C::kTmemCols);
@@ -171,8 +183,13 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             Unit u;
             while (ok && sc.next(p, u)) {
                 const int32_t ra = u.ta * kPairBM + static_cast<int32_t>(rank) * kBM;
-                // B rows of sub-tile s: u.tb * BN + s * kSubN + rank * kSubN / 2, kSubN / 2 of them
-                const int32_t rb = u.tb * BN + static_cast<int32_t>(rank) * (C::kSubN / 2);
+                // B rows of sub-tile s: u.col0 + s * kSubN + rank * kSubN / 2, kSubN / 2 of them
+                const int32_t rb = static_cast<int32_t>(u.col0) + static_cast<int32_t>(rank) * (C::kSubN / 2);
+                // a 384-wide unit: its second sub-tile is 128 wide, 64 rows per CTA
+                const bool narrow = kWide && u.w < BN;
+                const int32_t rb2 = static_cast<int32_t>(u.col0) + C::kSubN + static_cast<int32_t>(rank) * (kNarrowSubN / 2);
+                const uint32_t kb_bytes = narrow ? static_cast<uint32_t>(C::kABytes + C::kSubBBytes + C::kSubBBytes / 2)
+                                                 : static_cast<uint32_t>(C::kKbBytes);
                 for (int kb = u.kb0; kb < u.kb1; kb += KPS) {
                     const int n = (u.kb1 - kb < KPS) ? u.kb1 - kb : KPS;  // k-blocks in this stage
                     if (!mbar_wait_bounded(bar_empty(stage), phase ^ 1u, abort_flag, p.timeout_ns,
@@ -199,14 +216,19 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                         }
                     } else {
                         // the leader expects both CTAs' bytes on its own full barrier
-                        if (rank == 0) mbar_arrive_expect_tx(bar_full(stage), 2 * n * C::kKbBytes);
+                        if (rank == 0) mbar_arrive_expect_tx(bar_full(stage), 2 * n * kb_bytes);
                         const uint32_t leader_full = mapa_shared(bar_full(stage), 0);
                         for (int j = 0; j < n; ++j) {
                             tma_load_2d_pair(sA(stage) + j * C::kABytes, &tmA, leader_full, (kb + j) * kBKW, ra);
 #pragma unroll
-                            for (int sb = 0; sb < C::kNSub; ++sb)
-                                tma_load_2d_pair(sB(stage) + j * C::kBBytes + sb * C::kSubBBytes, &tmB, leader_full,
-                                                 (kb + j) * kBKW, rb + sb * C::kSubN);
+                            for (int sb = 0; sb < C::kNSub; ++sb) {
+                                if (kWide && sb == 1 && narrow)
+                                    tma_load_2d_pair(sB(stage) + j * C::kBBytes + sb * C::kSubBBytes, &tmB2, leader_full,
+                                                     (kb + j) * kBKW, rb2);
+                                else
+                                    tma_load_2d_pair(sB(stage) + j * C::kBBytes + sb * C::kSubBBytes, &tmB, leader_full,
+                                                     (kb + j) * kBKW, rb + sb * C::kSubN);
+                            }
                         }
                     }
                     ++fills;
@@ -234,6 +256,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             sc.init(p, pair, num_pairs);
             Unit u;
             while (ok && sc.next(p, u)) {
+                const bool narrow = kWide && u.w < BN;
                 for (int kc = u.kb0; ok && kc < u.kb1; kc += kChunkKb) {
                     const int kce = (u.kb1 - kc > kChunkKb) ? kc + kChunkKb : u.kb1;
                     if (!mbar_wait_bounded(bar_acce(buf), acc_phase ^ 1u, abort_flag, p.timeout_ns,
@@ -282,7 +305,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                                     for (int sb = 0; sb < C::kNSub; ++sb)
                                         mma_tf32_pair(d_tmem + static_cast<uint32_t>(sb * C::kSubN), a_hi + koff,
                                                       desc(sB(stage) + j * C::kBBytes + sb * C::kSubBBytes) + koff,
-                                                      kIdesc, acc);
+                                                      (kWide && sb == 1 && narrow) ? kIdescNarrow : kIdesc, acc);
                                 }
                             }
                         }
@@ -366,8 +389,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         const int half = (warp - 4) >> 2;
         const int r = q * 32 + lane;
         constexpr int kChunks = BN / 32;
-        constexpr int kHalf = (kChunks + 1) / 2;  // chunks per half
-        const int c_lo = half * kHalf;
+        constexpr int kHalf = (kChunks + 1) / 2;  // chunks per half (the most)
         EpiOut eo;
         eo.tmap = p.tma_out ? &tmOut : nullptr;
         eo.stage = reinterpret_cast<float*>(epi_stage + (warp - 4) * kEpiTileBytes);
@@ -381,9 +403,14 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         Unit u;
         bool ok = true;
         while (ok && sc.next(p, u)) {
-            const int64_t cols_left = (SWAP ? p.M : p.N) - static_cast<int64_t>(u.tb) * BN;
-            const int nchunks = static_cast<int>(cols_left >= BN ? kChunks : (cols_left + 31) / 32);
-            const int mine = nchunks - c_lo < 0 ? 0 : (nchunks - c_lo > kHalf ? kHalf : nchunks - c_lo);
+            // this unit's chunks (a 384-wide unit of a mixed plan has 12),
+            // split between the two halves of the epilogue warps
+            const int u_chunks = kWide ? u.w / 32 : kChunks;
+            const int u_half = kWide ? u_chunks / 2 : kHalf;
+            const int c_lo = half * u_half;
+            const int64_t cols_left = (SWAP ? p.M : p.N) - u.col0;
+            const int nchunks = static_cast<int>(cols_left >= u_chunks * 32 ? u_chunks : (cols_left + 31) / 32);
+            const int mine = nchunks - c_lo < 0 ? 0 : (nchunks - c_lo > u_half ? u_half : nchunks - c_lo);
             // This CTA's 128 rows of the pair tile, as a 128-row tile index.
             Unit uh = u;
             uh.ta = 2 * u.ta + static_cast<int>(rank);

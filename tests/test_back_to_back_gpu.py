@@ -6,7 +6,7 @@ late arrival would land in whichever CTA the SM runs next, in the middle of
 another launch's barriers, flags or tiles.  Here launches of different pair
 kernels (224-wide split tiles with one k-block per stage, the pool kind,
 512-wide tiles, swapped tiles split along K, 224-wide tiles of two k-blocks
-per stage) follow one another without pauses, many times over, so that each
+per stage, a plan of mixed 512- and 384-wide tiles) follow one another without pauses, many times over, so that each
 launch's successor on an SM has a different shared-memory layout.  Every
 repeat must end with a clean status and be bitwise equal to the first run of
 the same shape, which matches the oracle.
@@ -26,6 +26,7 @@ SHAPES = [
     (1024, 2048, 8192, "scale_hardtanh_gelu", "tile=256x512"),
     (64, 2048, 75 * 256, "swish_scale", "pair=1 swap=1"),
     (2560, 1024, 4096, "none", "kps=2"),
+    (2000, 260, 7000, "scale_hardtanh_gelu", "mix=74x512"),
 ]
 
 

@@ -9,7 +9,8 @@ stage tags, and the peer's epilogue the leader's accumulator tags, through
 distributed shared memory.  A mismatch, or a producer re-arming a stage whose
 phase already completed, records FLE_ERR_PROTOCOL in the device status word.
 These checks stand in for a race detector (compute-sanitizer is not
-available here).  Variants: the default plans (both kernels), the one-CTA
+available here).  Variants: the default plans (both kernels, a plan of
+mixed 512- and 384-wide pair tiles among them), the one-CTA
 kernel alone (FLE_PAIR=0) and under an even stream-K spread (FLE_SCHED=sk:
 short units, CTAs holding two shared tiles), the pair kernel under the same
 spread, and 256-wide pair tiles of one k-block per stage (FLE_PAIR_BN=256
@@ -40,7 +41,7 @@ bad, plans = [], []
 shapes = [(7, 36, 33, "none"), (100, 1056, 520, "swish_scale"), (16, 8192, 4096, "scale_hardtanh_gelu"),
           (300, 2048, 1000, "scale_hardtanh_gelu"), (520, 2080, 1500, "avgpool_gelu_scale_rowmax"),
           (1024, 1024, 8192, "avgpool_gelu_scale_rowmax"), (64, 2048, 75 * 256, "swish_scale"),
-          (600, 4096, 2300, "none")]
+          (600, 4096, 2300, "none"), (2000, 260, 7000, "scale_hardtanh_gelu")]
 for M, K, N, problem in shapes:
     for precision in ("tf32", "3xtf32"):
         x, W, b = synth.linear_inputs(M, K, N, seed=M + N, device="cuda")

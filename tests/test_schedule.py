@@ -76,9 +76,9 @@ def check_schedule(M, K, N, problem, precision, sms):
     for c, rows in enumerate(per_cta):
         partial_slots = []
         for r in rows:
-            t, ta, tb, kb0, kb1, partial, slot, first, last, slot_rule = (int(v) for v in r)
+            t, ta, tb, kb0, kb1, partial, slot, first, last, slot_rule, b0, bw = (int(v) for v in r)
             assert 0 <= kb0 < kb1 <= num_kb
-            cover[t].append((kb0, kb1, c, (ta, tb), partial, slot, first, last, slot_rule))
+            cover[t].append((kb0, kb1, c, (ta, tb, b0, bw), partial, slot, first, last, slot_rule))
             if partial:
                 partial_slots.append(slot)
                 assert slot == slot_rule
@@ -88,7 +88,14 @@ def check_schedule(M, K, N, problem, precision, sms):
     assert tiles == list(range(len(tiles)))
     tas = {e[3][0] for v in cover.values() for e in v}
     tbs = {e[3][1] for v in cover.values() for e in v}
-    assert len(tas) * len(tbs) == len(tiles)
+    if tbs == {-1}:
+        check_mixed_widths(M, N, cover, per_cta)
+    else:
+        assert len(tas) * len(tbs) == len(tiles)
+        # a uniform grid: tile tb starts at B row tb * width
+        widths = {e[3][3] for v in cover.values() for e in v}
+        assert len(widths) == 1
+        assert all(e[3][2] == e[3][1] * e[3][3] for v in cover.values() for e in v)
     # the tiles span exactly the operand rows (A side holds M, or N in the
     # swapped order, in tiles of 128 rows, or 256 rows on CTA pairs)
     a_rows = {math.ceil(M / 128), math.ceil(N / 128), math.ceil(M / 256), math.ceil(N / 256)}
@@ -118,18 +125,58 @@ def check_schedule(M, K, N, problem, precision, sms):
     assert max(load) - min(load) <= num_kb
 
 
+def check_mixed_widths(M, N, cover, per_cta):
+    # A plan of mixed tile widths (the 512-wide pair kernel): every 256-row
+    # panel of the output is cut into 512-wide tiles from column 0, then
+    # 384-wide ones, which together cover [0, N) once (the last may reach
+    # past N); at most one tile of each width per pair, all tiles whole.
+    assert M > 128
+    grid = len(per_cta)
+    panels = defaultdict(list)
+    for t, units in cover.items():
+        assert len(units) == 1 and units[0][4] == 0
+        ta, tb, b0, bw = units[0][3]
+        panels[ta].append((b0, bw))
+    assert sorted(panels) == list(range(math.ceil(M / 256)))
+    for ta, tl in panels.items():
+        tl.sort()
+        pos = 0
+        for b0, bw in tl:
+            assert b0 == pos and bw in (512, 384)
+            pos += bw
+        assert pos >= N and tl[-1][0] < N
+        ws = [bw for _, bw in tl]
+        assert ws == sorted(ws, reverse=True)  # 512-wide first
+    n512 = sum(1 for tl in panels.values() for _, bw in tl if bw == 512)
+    n384 = sum(1 for tl in panels.values() for _, bw in tl if bw == 384)
+    assert n512 <= grid and n384 <= grid
+    for rows in per_cta:
+        ws = [int(r[11]) for r in rows]
+        assert ws.count(512) <= 1 and ws.count(384) <= 1
+        if len(ws) == 2:
+            assert ws == [512, 384]  # the wide tile first
+
+
 def test_headline_shape_plans():
-    # 2048x8192x8192 in TF32 runs 256x512 tiles on CTA pairs (two 256-wide
-    # MMAs sharing each x tile): 128 tiles on the 74 pairs of 148 SMs, two
-    # waves of whole tiles.  In 3xTF32 (no wide tiles) it runs 256x256 tiles:
-    # 3.46 waves, three of whole tiles and the 34 tiles of the last wave split
-    # in two k-aligned halves on 68 pairs.
+    # 2048x8192x8192 in TF32 runs 256-row tiles on CTA pairs, of mixed
+    # widths: 128 tiles 512 wide (two 256-wide MMAs sharing each x tile)
+    # would be two waves on the 74 pairs of 148 SMs, the second of 54; the
+    # plan runs one wave of 74 tiles 512 wide and one of 73 tiles 384 wide
+    # (a 256-wide and a 128-wide MMA), each pair at most one of each.  In
+    # 3xTF32 (no wide tiles) it runs 256x256 tiles: 3.46 waves, three of whole
+    # tiles and the 34 tiles of the last wave split in two k-aligned halves
+    # on 68 pairs.
     desc = fle.desc_for("scale_hardtanh_gelu", "tf32")
     grid, per_cta = collect(2048, 8192, 8192, desc, 148)
-    assert grid == 74 and _tiles(per_cta) == 128
-    assert all(int(r[5]) == 0 for rows in per_cta for r in rows)
-    load = [sum(int(r[4]) - int(r[3]) for r in rows) for rows in per_cta]
-    assert sum(load) == 128 * 256 and sorted(set(load)) == [256, 512]
+    assert grid == 74 and _tiles(per_cta) == 74 + 73
+    units = [r for rows in per_cta for r in rows]
+    assert all(int(r[5]) == 0 for r in units)
+    assert sum(1 for r in units if int(r[11]) == 512) == 74
+    assert sum(1 for r in units if int(r[11]) == 384) == 73
+    # columns per pair: 512 + 384 on 73 pairs, 512 on one
+    cols = sorted(sum(int(r[11]) for r in rows) for rows in per_cta)
+    assert cols == [512] + [896] * 73
+    check_schedule(2048, 8192, 8192, "scale_hardtanh_gelu", "tf32", 148)
     grid3, per3 = collect(2048, 8192, 8192, fle.desc_for("scale_hardtanh_gelu", "3xtf32"), 148)
     assert grid3 == 74 and _tiles(per3) == 256
     load = [sum(int(r[4]) - int(r[3]) for r in rows) for rows in per3]
@@ -212,8 +259,27 @@ def test_pair_tile_width_fills_the_waves():
     grid, per = collect(256, 8192, 8192, d, 148)
     assert grid == 74 and _tiles(per) == 37
     assert all(len(rows) == 1 and int(rows[0][5]) == 1 for rows in per)
+    # 2048 x 8192 x 8192: 512 wide, cut into mixed widths (see the headline test)
     grid, per = collect(2048, 8192, 8192, d, 148)
-    assert _tiles(per) == 8 * 16
+    assert {int(r[11]) for rows in per for r in rows} == {512, 384}
+
+
+def test_mixed_widths_only_where_they_shorten_the_plan():
+    # The mixed cut is taken for 512-wide plans of more than one wave that
+    # it shortens: not for 4096 x 8192 x 8192 (3.5 waves: three whole and
+    # one split in two), 1024 x 8192 x 8192 (one wave) or 2304 x 2048 x 8192
+    # (144 tiles, no cut fits); yes for 3584 x 128 x 4096 (112 tiles of 512:
+    # 74 of 512 and 52 of 384), 4096 x 128 x 3584 (16 panels) and the ragged
+    # 2000 x 260 x 7000.
+    d = fle.desc_for("none", "tf32")
+    for M, K, N in [(4096, 8192, 8192), (1024, 8192, 8192), (2304, 2048, 8192)]:
+        _, per = collect(M, K, N, d, 148)
+        assert all(int(r[2]) >= 0 for rows in per for r in rows), (M, K, N)
+    for M, K, N, wide, narrow in [(3584, 128, 4096, 74, 52), (4096, 128, 3584, 74, 54), (2000, 260, 7000, 74, 52)]:
+        grid, per = collect(M, K, N, d, 148)
+        ws = [int(r[11]) for rows in per for r in rows]
+        assert ws.count(512) == wide and (narrow is None or ws.count(384) == narrow), (M, K, N)
+        check_schedule(M, K, N, "none", "tf32", 148)
 
 
 def test_uneven_last_wave_spreads_only_in_3xtf32():

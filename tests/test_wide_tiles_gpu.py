@@ -9,6 +9,14 @@ when it is cheaper than 256 or 224 columns per tile (2048, 4096 and 1024 x
 along K; and, with the width forced (FLE_PAIR_BN=512, read once per process,
 hence the subprocess), small ragged shapes of every epilogue kind, both
 finisher branches of split tiles (bitwise equal) and the oracle.
+
+The same kernel runs the mixed-width plans: one wave of 512-wide tiles and
+one of 384-wide tiles (a 256-wide and a 128-wide MMA sharing the A tile,
+whose 64 weight rows per CTA come through a second tensor map), cut per
+256-row panel.  Covered: ragged M, K and N, 8 to 16 panels, every epilogue
+kind, against the oracle on rows from every panel, and bitwise against the
+uniform 512-wide plan of the same inputs (FLE_MIX=0): an output element gets
+the same MMA chain over the same k-blocks in either plan.
 """
 import os
 import subprocess
@@ -110,3 +118,60 @@ def test_forced_wide_tiles_small_shapes(fle):
                        timeout=900)
     assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-4000:]
     assert r.stdout.count("PLAN tile=256x512") == 5
+
+
+MIXED = [
+    (2000, 260, 7000, "scale_hardtanh_gelu"),        # ragged M, K and N: 74 + 52 tiles
+    (3584, 128, 4096, "swish_scale"),                # 14 panels
+    (4096, 128, 3584, "none"),                       # 16 panels
+    (2048, 128, 7000, "avgpool_gelu_scale_rowmax"),  # pool windows across 384-wide tiles
+]
+
+
+def _panel_rows(M, seed):
+    # the first and last row of every 256-row panel and 64 more at random
+    rows = set()
+    for p0 in range(0, M, 256):
+        rows.update((p0, min(p0 + 255, M - 1)))
+    rows.update(int(r) for r in synth.sample_rows(M, 64, seed=seed))
+    return np.array(sorted(rows))
+
+
+_UNIFORM_SCRIPT = r"""
+import sys, numpy as np, torch
+import reduction_epilogue_b200 as fle
+from reduction_epilogue_b200 import synth
+fle.load()
+M, K, N, problem, path = sys.argv[1], sys.argv[2], sys.argv[3], sys.argv[4], sys.argv[5]
+M, K, N = int(M), int(K), int(N)
+plan = fle.plan_string(M, K, N, fle.desc_for(problem, "tf32"))
+assert "mix=" not in plan and "tile=256x512" in plan, plan
+x, W, b = synth.linear_inputs(M, K, N, seed=M + N + 7, device="cuda")
+out = fle.linear_epilogue(x, W, b, problem, "tf32")
+torch.cuda.synchronize()
+assert fle.device_status() == 0
+np.save(path, out.cpu().numpy())
+print("PLAN", plan)
+"""
+
+
+@pytest.mark.parametrize("M,K,N,problem", MIXED)
+def test_mixed_width_plans(fle, M, K, N, problem, tmp_path):
+    d = fle.desc_for(problem, "tf32")
+    plan = fle.plan_string(M, K, N, d)
+    assert "tile=256x512 pair=1" in plan and " mix=74x512+" in plan and "sk_tiles=0 " in plan, plan
+    x, W, b = synth.linear_inputs(M, K, N, seed=M + N + 7, device="cuda")
+    out = fle.linear_epilogue(x, W, b, problem, "tf32")
+    torch.cuda.synchronize()
+    assert fle.device_status() == 0
+    pool = problem == "avgpool_gelu_scale_rowmax"
+    rows = np.arange(M) if pool else _panel_rows(M, seed=9)
+    ref = oracle.forward_rows(x.cpu().numpy(), W.cpu().numpy(), b.cpu().numpy(), rows=rows, **oracle.PROBLEMS[problem])
+    _close(out.cpu().numpy()[rows], ref, f"{problem} {M}x{K}x{N} {plan}")
+    # the uniform 512-wide plan of the same inputs, in a fresh process
+    path = str(tmp_path / "uniform.npy")
+    env = dict(os.environ, FLE_MIX="0", PYTHONPATH=ROOT)
+    r = subprocess.run([sys.executable, "-c", _UNIFORM_SCRIPT, str(M), str(K), str(N), problem, path], cwd=ROOT,
+                       env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+    assert np.array_equal(np.load(path), out.cpu().numpy()), "mixed and uniform plans differ"
