@@ -526,6 +526,37 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
     return v;
 }
 
+// 3xTF32 low parts of one ring stage, by the 64 threads of the two split
+// warps (ct = 0..63): for each of the stage's kVec float4, lo = x - hi with hi
+// = x with the low 13 mantissa bits cleared (a TF32 value; x - hi is exact in
+// fp32).  A batch of loads is issued before its stores: the raw and low
+// halves of a stage do not overlap, and without that (or the restrict
+// qualifiers) each store would have to complete before the next load issues,
+// serialising the stage on the shared-memory latency.
+constexpr int kSplitBatch = 8;  // float4 per thread in flight (measured: 8 = 16 > 32)
+
+template <int kVec>
+__device__ __forceinline__ void split_lo_parts(const float4* __restrict__ x4, float4* __restrict__ lo4, int ct) {
+    static_assert(kVec % 64 == 0, "whole float4 rows for the 64 split threads");
+    constexpr int kPer = kVec / 64;
+#pragma unroll
+    for (int b0 = 0; b0 < kPer; b0 += kSplitBatch) {
+        float4 v[kSplitBatch];
+#pragma unroll
+        for (int u = 0; u < kSplitBatch; ++u)
+            if (b0 + u < kPer) v[u] = x4[ct + 64 * (b0 + u)];
+#pragma unroll
+        for (int u = 0; u < kSplitBatch; ++u)
+            if (b0 + u < kPer) {
+                const float4 x = v[u];
+                lo4[ct + 64 * (b0 + u)] = make_float4(x.x - __uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u),
+                                                      x.y - __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u),
+                                                      x.z - __uint_as_float(__float_as_uint(x.z) & 0xFFFFE000u),
+                                                      x.w - __uint_as_float(__float_as_uint(x.w) & 0xFFFFE000u));
+            }
+    }
+}
+
 // Barrier among the eight epilogue warps only (named barrier 1, 256 threads).
 __device__ __forceinline__ void epilogue_bar_sync() {
     asm volatile("bar.sync 1, 256;" ::: "memory");
@@ -690,8 +721,10 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
                 for (int kb = kc; kb < kce; kb += KPS) {
                     const int n = (kce - kb < KPS) ? kce - kb : KPS;  // k-blocks in this stage
-                    const uint32_t wbar = (PREC == kPrec3xTF32) ? bar_conv(stage) : bar_full(stage);
-                    if (!mbar_wait_bounded(wbar, phase, abort_flag, p.timeout_ns, kWhereMmaFull)) {
+                    // hi x hi reads only the copied tiles: it runs as soon as
+                    // they land (3xTF32: while the split warps write the low
+                    // parts), the products with a low part after the split
+                    if (!mbar_wait_bounded(bar_full(stage), phase, abort_flag, p.timeout_ns, kWhereMmaFull)) {
                         ok = false;
                         break;
                     }
@@ -705,14 +738,25 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                             // advance 8 fp32 = 32 bytes along K inside the swizzle atom
                             const uint64_t koff = static_cast<uint64_t>(k * 2);
                             const uint32_t acc = (kb > kc || j > 0 || k > 0) ? 1u : 0u;
-                            if constexpr (PREC == kPrec3xTF32) {
-                                const uint64_t a_lo = smem_desc_sw128(sA(stage) + C::kLoadBytes + j * C::kABytes);
-                                const uint64_t b_lo = smem_desc_sw128(sB(stage) + C::kLoadBytes + j * C::kBBytes);
-                                mma_tf32(d_tmem, a_lo + koff, b_hi + koff, kIdesc, acc);
+                            mma_tf32(d_tmem, a_hi + koff, b_hi + koff, kIdesc, acc);
+                        }
+                    }
+                    if constexpr (PREC == kPrec3xTF32) {
+                        if (!mbar_wait_bounded(bar_conv(stage), phase, abort_flag, p.timeout_ns, kWhereMmaFull)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after_sync();
+                        for (int j = 0; j < n; ++j) {
+                            const uint64_t a_hi = smem_desc_sw128(sA(stage) + j * C::kABytes);
+                            const uint64_t b_hi = smem_desc_sw128(sB(stage) + j * C::kBBytes);
+                            const uint64_t a_lo = smem_desc_sw128(sA(stage) + C::kLoadBytes + j * C::kABytes);
+                            const uint64_t b_lo = smem_desc_sw128(sB(stage) + C::kLoadBytes + j * C::kBBytes);
+#pragma unroll
+                            for (int k = 0; k < kBK / kUmmaK; ++k) {
+                                const uint64_t koff = static_cast<uint64_t>(k * 2);
+                                mma_tf32(d_tmem, a_lo + koff, b_hi + koff, kIdesc, 1u);
                                 mma_tf32(d_tmem, a_hi + koff, b_lo + koff, kIdesc, 1u);
-                                mma_tf32(d_tmem, a_hi + koff, b_hi + koff, kIdesc, 1u);
-                            } else {
-                                mma_tf32(d_tmem, a_hi + koff, b_hi + koff, kIdesc, acc);
                             }
                         }
                     }
@@ -759,15 +803,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     // operand-conversion test).
                     const float4* x4 = reinterpret_cast<const float4*>(smem + stage * C::kStageBytes);
                     float4* lo4 = reinterpret_cast<float4*>(smem + stage * C::kStageBytes + C::kLoadBytes);
-                    constexpr int kVec = C::kLoadBytes / 16;
-#pragma unroll 4
-                    for (int i = ct; i < kVec; i += 64) {
-                        const float4 x = x4[i];
-                        lo4[i] = make_float4(x.x - __uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u),
-                                             x.y - __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u),
-                                             x.z - __uint_as_float(__float_as_uint(x.z) & 0xFFFFE000u),
-                                             x.w - __uint_as_float(__float_as_uint(x.w) & 0xFFFFE000u));
-                    }
+                    split_lo_parts<C::kLoadBytes / 16>(x4, lo4, ct);
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar_conv(stage));

@@ -363,15 +363,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     }
                     const float4* x4 = reinterpret_cast<const float4*>(smem + stage * C::kStageBytes);
                     float4* lo4 = reinterpret_cast<float4*>(smem + stage * C::kStageBytes + C::kLoadBytes);
-                    constexpr int kVec = C::kLoadBytes / 16;
-#pragma unroll 4
-                    for (int i = ct; i < kVec; i += 64) {
-                        const float4 x = x4[i];
-                        lo4[i] = make_float4(x.x - __uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u),
-                                             x.y - __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u),
-                                             x.z - __uint_as_float(__float_as_uint(x.z) & 0xFFFFE000u),
-                                             x.w - __uint_as_float(__float_as_uint(x.w) & 0xFFFFE000u));
-                    }
+                    split_lo_parts<C::kLoadBytes / 16>(x4, lo4, ct);
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) mbar_arrive_cluster(mapa_shared(bar_split(stage), 0));
