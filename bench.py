@@ -436,10 +436,12 @@ def run_fle(args, name, dist_ctx, precision=None, brief=False):
         def step():
             fle.forward(x, W, b, out, desc, workspace=ws, workspace_bytes=ws_bytes, stream=stream)
     # our kernels per call: the GEMM, a prep kernel when the plan splits K or
-    # the kind is (c), and the weight pooling of the per-call pool-fold
-    plan_sk = "sk_tiles=0 " not in fle.plan_string(*plan_shape)
+    # the kind is (c), the 3xTF32 pre-pass that writes x's low parts, and the
+    # weight pooling of the per-call pool-fold
+    plan_text = fle.plan_string(*plan_shape)
+    plan_sk = "sk_tiles=0 " not in plan_text
     launches_per_step = (1 + (1 if (problem == "avgpool_gelu_scale_rowmax" or plan_sk) else 0)
-                         + (1 if variant == "poolfold" else 0))
+                         + (1 if " xlo=mem" in plan_text else 0) + (1 if variant == "poolfold" else 0))
 
     input_bytes = 4 * (M * K + N * K + N)
     if variant == "poolfold_cached":

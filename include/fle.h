@@ -26,7 +26,8 @@
  *
  * All entry points are plain C: host scalars, and device pointers to fp32
  * data that the caller owns.  Nothing here allocates device memory; scratch
- * for split-K comes from the caller (fle_workspace_size / workspace).
+ * (split-K partials; in 3xTF32 the low parts of x) comes from the caller
+ * (fle_workspace_size / workspace).
  */
 #ifndef FLE_H
 #define FLE_H
@@ -99,7 +100,7 @@ enum {
                                 out / b not 4-byte aligned                   */
     FLE_ERR_DESC = 4,        /* unknown kind/precision/flag, non-finite scale
                                 or clamp, clamp_lo > clamp_hi, unsupported pool */
-    FLE_ERR_WORKSPACE = 5,   /* workspace smaller than fle_workspace_size()  */
+    FLE_ERR_WORKSPACE = 5,   /* workspace smaller than fle_workspace_size_min() */
     FLE_ERR_ARCH = 6,        /* current device is not sm_100 (B200)          */
     FLE_ERR_CUDA = 7,        /* a CUDA runtime/driver call failed            */
     FLE_ERR_TIMEOUT = 8,     /* a device-side bounded wait expired           */
@@ -120,10 +121,13 @@ enum {
  *   out     device, fp32 [M,N] row-major for (a), (b) and NONE; fp32 [M] for
  *           (c).  Must not overlap x, W, b or the workspace.
  *   workspace, workspace_bytes
- *           device scratch of at least fle_workspace_size(M,K,N,desc) bytes,
- *           256-byte aligned (may be NULL/0 when that size is 0).  Its contents
- *           on entry are ignored; it must not be used by another call that
- *           runs concurrently on the GPU.
+ *           device scratch of fle_workspace_size(M,K,N,desc) bytes, or at
+ *           least fle_workspace_size_min() bytes (then a plan that fits runs:
+ *           in 3xTF32 the low parts of x are computed inside the GEMM instead
+ *           of once per call into the workspace), 256-byte aligned (may be
+ *           NULL/0 when that size is 0).  Its contents on entry are ignored;
+ *           it must not be used by another call that runs concurrently on the
+ *           GPU.
  *   stream  a cudaStream_t (NULL = the legacy default stream)
  *
  * Returns FLE_OK once the work is enqueued (no host synchronisation).
@@ -179,10 +183,17 @@ int fle_forward_pooled(const float* x, const float* W, const float* b,
                        const fle_epilogue_desc* desc, float* out,
                        void* workspace, size_t workspace_bytes, void* stream);
 
-/* Bytes of caller workspace fle_forward needs for these arguments (0 when
- * the chosen schedule needs none).  Returns 0 for invalid arguments too;
- * fle_forward then reports the argument error. */
+/* Bytes of caller workspace for the fastest plan of these arguments (0 when
+ * the plan needs none): split-K partial tiles and arrival counters, and in
+ * 3xTF32 the low parts of x (M x K fp32, written by a pre-pass so that the
+ * GEMM splits only W).  Returns 0 for invalid arguments too; fle_forward then
+ * reports the argument error. */
 size_t fle_workspace_size(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* desc);
+
+/* The least workspace fle_forward accepts for these arguments: the plan
+ * without x's low parts in memory (equal to fle_workspace_size() in TF32).
+ * Same results bit for bit; 3xTF32 runs slower with it. */
+size_t fle_workspace_size_min(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* desc);
 
 /* Static text for a status code; never NULL. */
 const char* fle_status_string(int status);
@@ -224,11 +235,12 @@ int fle_plan_units(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* des
  * latency-critical loop in which cudaMalloc/cudaFree would synchronise the
  * device and stall every other stream.  This entry point needs no workspace
  * argument and allocates nothing: the scratch that fle_forward takes from
- * `workspace` (stream-K partial tiles and arrival counters) comes from one
- * static device array of FLE_NOALLOC_SCRATCH_BYTES (40 MiB) inside the
- * library.  Every plan on a 148-SM B200 needs at most about 37 MiB; a plan
- * that would need more is rejected with FLE_ERR_WORKSPACE before anything is
- * enqueued.  The caller still owns and passes x, W, b and out, with the same
+ * `workspace` (stream-K partial tiles and arrival counters; 3xTF32's low
+ * parts of x when they fit as well) comes from one static device array of
+ * FLE_NOALLOC_SCRATCH_BYTES (40 MiB) inside the library.  Every plan on a
+ * 148-SM B200 fits with x's low parts computed inside the GEMM
+ * (fle_workspace_size_min: at most about 37 MiB); a plan that would need more
+ * is rejected with FLE_ERR_WORKSPACE before anything is enqueued.  The caller still owns and passes x, W, b and out, with the same
  * layout, alignment and error rules as fle_forward.
  *
  * The first call on each device looks up the array's device address (with

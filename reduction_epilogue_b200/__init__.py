@@ -16,7 +16,7 @@ import os
 __all__ = [
     "EPI_SCALE_HARDTANH_GELU", "EPI_SWISH_SCALE", "EPI_AVGPOOL_GELU_SCALE_ROWMAX", "EPI_NONE",
     "PREC_3XTF32", "PREC_TF32", "EpilogueDesc", "FleError", "desc_for", "forward",
-    "workspace_size", "device_status", "plan_string", "plan_units", "pool_weights",
+    "workspace_size", "workspace_size_min", "device_status", "plan_string", "plan_units", "pool_weights",
     "workspace_size_pooled", "forward_pooled", "linear_epilogue", "library_path", "load",
     "PROBLEMS",
 ]
@@ -99,6 +99,8 @@ def load():
     lib.fle_forward.restype = ctypes.c_int
     lib.fle_workspace_size.argtypes = [i64, i64, i64, ctypes.POINTER(EpilogueDesc)]
     lib.fle_workspace_size.restype = sz
+    lib.fle_workspace_size_min.argtypes = [i64, i64, i64, ctypes.POINTER(EpilogueDesc)]
+    lib.fle_workspace_size_min.restype = sz
     lib.fle_status_string.argtypes = [ctypes.c_int]
     lib.fle_status_string.restype = ctypes.c_char_p
     lib.fle_device_status.argtypes = [vp]
@@ -185,6 +187,10 @@ def _check_tensor(name, t, shape):
 
 def workspace_size(M: int, K: int, N: int, desc: EpilogueDesc) -> int:
     return int(load().fle_workspace_size(M, K, N, ctypes.byref(desc)))
+
+
+def workspace_size_min(M: int, K: int, N: int, desc: EpilogueDesc) -> int:
+    return int(load().fle_workspace_size_min(M, K, N, ctypes.byref(desc)))
 
 
 def plan_string(M: int, K: int, N: int, desc: EpilogueDesc) -> str:

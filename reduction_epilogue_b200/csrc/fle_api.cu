@@ -171,6 +171,10 @@ struct Plan {
     int mix_wide = 0, mix_narrow = 0;
     unsigned char mix_a[fle::kMaxMixPanels] = {};
     unsigned char mix_b[fle::kMaxMixPanels] = {};
+    // 3xTF32: the low parts of x written once into the workspace (at
+    // lo_offset, M x K fp32) by a pre-pass and copied with the tiles
+    bool lo_mem = false;
+    size_t lo_offset = 0;
 };
 
 // Ring depth of the single-CTA kernel (mirrors Cfg::kStages).
@@ -225,6 +229,15 @@ int pair_bn_override() {
         return (n == fle::kPairBN || n == fle::kPairBNNarrow || n == fle::kPairBNWide) ? n : 0;
     }();
     return v;
+}
+
+// FLE_LO_MEM=0 keeps 3xTF32's low parts of x inside the GEMM (comparisons).
+bool lo_mem_disabled() {
+    static bool off = [] {
+        const char* e = std::getenv("FLE_LO_MEM");
+        return e && e[0] == '0';
+    }();
+    return off;
 }
 
 // FLE_MIX=0 keeps the 512-wide plans on a uniform grid (comparisons).
@@ -309,7 +322,11 @@ double plan_waves(int64_t T, int64_t G, int num_kb, int64_t min_iters, bool spre
 }
 
 // sms: SMs of the device; pairs: co-resident CTA pairs of the pair kernel.
-Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int sms, int pairs) {
+// lo_mem: 3xTF32 plans may keep x's low parts in the workspace (the fastest
+// plan); without it their split warps compute them for every tile.
+Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int sms, int pairs,
+               bool lo_mem = true);
+Plan make_plan_core(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int sms, int pairs) {
     Plan pl;
     pl.prec = (d->precision == FLE_PREC_3XTF32) ? fle::kPrec3xTF32 : fle::kPrecTF32;
     pl.swap = (M <= 128) && d->kind != FLE_EPI_AVGPOOL_GELU_SCALE_ROWMAX;
@@ -479,12 +496,27 @@ Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int 
     return pl;
 }
 
+// 3xTF32: x's low parts are split once per call into the workspace, except
+// for skinny swapped shapes (M <= 64), where x is a small part of each stage
+// and the pre-pass does not pay (measured no faster at M = 16).  Measured
+// with the low parts in memory: 2048 x 8192 x 8192 1358 -> ~1066 us of GEMM,
+// 128 x 32768 x 32768 1766 -> ~1565 us, M = 256 239 -> ~198 us.
+Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int sms, int pairs, bool lo_mem) {
+    Plan pl = make_plan_core(M, K, N, d, sms, pairs);
+    if (lo_mem && pl.prec == fle::kPrec3xTF32 && K > 0 && !(pl.swap && M <= 64) && !lo_mem_disabled()) {
+        pl.lo_mem = true;
+        pl.lo_offset = (pl.ws_bytes + 255) & ~size_t(255);
+        pl.ws_bytes = pl.lo_offset + static_cast<size_t>(M) * static_cast<size_t>(K) * sizeof(float);
+    }
+    return pl;
+}
+
 // after_prep: the previous kernel in the stream is this call's prep kernel,
 // which writes nothing the GEMM reads before griddep_wait(); the GEMM is then
 // launched with programmatic stream serialization and starts during it.
 template <int BN, int PREC, bool SWAP, int KPS>
-cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to, const KParams& p,
-                        int grid, bool after_prep, cudaStream_t st) {
+cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& txlo, const CUtensorMap& to,
+                        const KParams& p, int grid, bool after_prep, cudaStream_t st) {
     using C = fle::Cfg<BN, PREC, SWAP, KPS>;
     auto kern = fle::fle_gemm_kernel<BN, PREC, SWAP, KPS>;
     static std::atomic<bool> attr_set[kMaxDevices] = {};
@@ -505,14 +537,15 @@ cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUte
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = after_prep ? 1 : 0;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, to, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, txlo, to, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
 template <int PREC, int KPS, int BN = fle::kPairBN, bool SWAP = false>
 cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb2,
-                             const CUtensorMap& to, const KParams& p, int pairs, bool after_prep, cudaStream_t st) {
+                             const CUtensorMap& txlo, const CUtensorMap& to, const KParams& p, int pairs,
+                             bool after_prep, cudaStream_t st) {
     using C = fle::PairCfg<PREC, KPS, BN, SWAP>;
     auto kern = fle::fle_gemm_pair_kernel<PREC, KPS, BN, SWAP>;
     static std::atomic<bool> attr_set[kMaxDevices] = {};
@@ -537,36 +570,38 @@ cudaError_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = after_prep ? 2 : 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tb2, to, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tb2, txlo, to, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
 // tb2: the 64-row boxes of B for the 384-wide tiles of a mixed plan (else tb).
+// txlo: 3xTF32 with x's low parts in memory, their tensor map (else ta).
 cudaError_t dispatch(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb2,
-                     const CUtensorMap& to, const KParams& p, bool after_prep, cudaStream_t st) {
+                     const CUtensorMap& txlo, const CUtensorMap& to, const KParams& p, bool after_prep,
+                     cudaStream_t st) {
     using namespace fle;
     const bool tf32 = pl.prec == kPrecTF32;
     const bool two = pl.kps == 2;  // TF32 only
     if (pl.pair && !pl.swap && pl.bn == kPairBNWide)
-        return launch_gemm_pair<kPrecTF32, 1, kPairBNWide>(ta, tb, tb2, to, p, pl.grid, after_prep, st);
+        return launch_gemm_pair<kPrecTF32, 1, kPairBNWide>(ta, tb, tb2, txlo, to, p, pl.grid, after_prep, st);
     if (pl.pair && !pl.swap && pl.bn == kPairBNNarrow) {
-        if (!tf32) return launch_gemm_pair<kPrec3xTF32, 1, kPairBNNarrow>(ta, tb, tb2, to, p, pl.grid, after_prep, st);
-        return two ? launch_gemm_pair<kPrecTF32, 2, kPairBNNarrow>(ta, tb, tb2, to, p, pl.grid, after_prep, st)
-                   : launch_gemm_pair<kPrecTF32, 1, kPairBNNarrow>(ta, tb, tb2, to, p, pl.grid, after_prep, st);
+        if (!tf32) return launch_gemm_pair<kPrec3xTF32, 1, kPairBNNarrow>(ta, tb, tb2, txlo, to, p, pl.grid, after_prep, st);
+        return two ? launch_gemm_pair<kPrecTF32, 2, kPairBNNarrow>(ta, tb, tb2, txlo, to, p, pl.grid, after_prep, st)
+                   : launch_gemm_pair<kPrecTF32, 1, kPairBNNarrow>(ta, tb, tb2, txlo, to, p, pl.grid, after_prep, st);
     }
     if (pl.pair && !pl.swap) {
-        if (!tf32) return launch_gemm_pair<kPrec3xTF32, 1>(ta, tb, tb2, to, p, pl.grid, after_prep, st);
-        return two ? launch_gemm_pair<kPrecTF32, 2>(ta, tb, tb2, to, p, pl.grid, after_prep, st)
-                   : launch_gemm_pair<kPrecTF32, 1>(ta, tb, tb2, to, p, pl.grid, after_prep, st);
+        if (!tf32) return launch_gemm_pair<kPrec3xTF32, 1>(ta, tb, tb2, txlo, to, p, pl.grid, after_prep, st);
+        return two ? launch_gemm_pair<kPrecTF32, 2>(ta, tb, tb2, txlo, to, p, pl.grid, after_prep, st)
+                   : launch_gemm_pair<kPrecTF32, 1>(ta, tb, tb2, txlo, to, p, pl.grid, after_prep, st);
     }
     if (pl.pair) {
         switch (pl.bn) {
 #define FLE_PAIR_SWAP_CASE(bn)                                                                             \
     case bn:                                                                                               \
-        if (!tf32) return launch_gemm_pair<kPrec3xTF32, 1, bn, true>(ta, tb, tb2, to, p, pl.grid, after_prep, st); \
-        return two ? launch_gemm_pair<kPrecTF32, 2, bn, true>(ta, tb, tb2, to, p, pl.grid, after_prep, st)      \
-                   : launch_gemm_pair<kPrecTF32, 1, bn, true>(ta, tb, tb2, to, p, pl.grid, after_prep, st);
+        if (!tf32) return launch_gemm_pair<kPrec3xTF32, 1, bn, true>(ta, tb, tb2, txlo, to, p, pl.grid, after_prep, st); \
+        return two ? launch_gemm_pair<kPrecTF32, 2, bn, true>(ta, tb, tb2, txlo, to, p, pl.grid, after_prep, st)      \
+                   : launch_gemm_pair<kPrecTF32, 1, bn, true>(ta, tb, tb2, txlo, to, p, pl.grid, after_prep, st);
             FLE_PAIR_SWAP_CASE(32)
             FLE_PAIR_SWAP_CASE(64)
             FLE_PAIR_SWAP_CASE(128)
@@ -576,23 +611,23 @@ cudaError_t dispatch(const Plan& pl, const CUtensorMap& ta, const CUtensorMap& t
     }
     if (!pl.swap) {
         if (tf32 && pl.bn == 256)
-            return two ? launch_gemm<256, kPrecTF32, false, 2>(ta, tb, to, p, pl.grid, after_prep, st)
-                       : launch_gemm<256, kPrecTF32, false, 1>(ta, tb, to, p, pl.grid, after_prep, st);
-        if (!tf32 && pl.bn == 128) return launch_gemm<128, kPrec3xTF32, false, 1>(ta, tb, to, p, pl.grid, after_prep, st);
+            return two ? launch_gemm<256, kPrecTF32, false, 2>(ta, tb, txlo, to, p, pl.grid, after_prep, st)
+                       : launch_gemm<256, kPrecTF32, false, 1>(ta, tb, txlo, to, p, pl.grid, after_prep, st);
+        if (!tf32 && pl.bn == 128) return launch_gemm<128, kPrec3xTF32, false, 1>(ta, tb, txlo, to, p, pl.grid, after_prep, st);
     } else {
         switch (pl.bn) {
             case 32:
-                if (!tf32) return launch_gemm<32, kPrec3xTF32, true, 1>(ta, tb, to, p, pl.grid, after_prep, st);
-                return two ? launch_gemm<32, kPrecTF32, true, 2>(ta, tb, to, p, pl.grid, after_prep, st)
-                           : launch_gemm<32, kPrecTF32, true, 1>(ta, tb, to, p, pl.grid, after_prep, st);
+                if (!tf32) return launch_gemm<32, kPrec3xTF32, true, 1>(ta, tb, txlo, to, p, pl.grid, after_prep, st);
+                return two ? launch_gemm<32, kPrecTF32, true, 2>(ta, tb, txlo, to, p, pl.grid, after_prep, st)
+                           : launch_gemm<32, kPrecTF32, true, 1>(ta, tb, txlo, to, p, pl.grid, after_prep, st);
             case 64:
-                if (!tf32) return launch_gemm<64, kPrec3xTF32, true, 1>(ta, tb, to, p, pl.grid, after_prep, st);
-                return two ? launch_gemm<64, kPrecTF32, true, 2>(ta, tb, to, p, pl.grid, after_prep, st)
-                           : launch_gemm<64, kPrecTF32, true, 1>(ta, tb, to, p, pl.grid, after_prep, st);
+                if (!tf32) return launch_gemm<64, kPrec3xTF32, true, 1>(ta, tb, txlo, to, p, pl.grid, after_prep, st);
+                return two ? launch_gemm<64, kPrecTF32, true, 2>(ta, tb, txlo, to, p, pl.grid, after_prep, st)
+                           : launch_gemm<64, kPrecTF32, true, 1>(ta, tb, txlo, to, p, pl.grid, after_prep, st);
             case 128:
-                if (!tf32) return launch_gemm<128, kPrec3xTF32, true, 1>(ta, tb, to, p, pl.grid, after_prep, st);
-                return two ? launch_gemm<128, kPrecTF32, true, 2>(ta, tb, to, p, pl.grid, after_prep, st)
-                           : launch_gemm<128, kPrecTF32, true, 1>(ta, tb, to, p, pl.grid, after_prep, st);
+                if (!tf32) return launch_gemm<128, kPrec3xTF32, true, 1>(ta, tb, txlo, to, p, pl.grid, after_prep, st);
+                return two ? launch_gemm<128, kPrecTF32, true, 2>(ta, tb, txlo, to, p, pl.grid, after_prep, st)
+                           : launch_gemm<128, kPrecTF32, true, 1>(ta, tb, txlo, to, p, pl.grid, after_prep, st);
             default: break;
         }
     }
@@ -636,6 +671,10 @@ int plan_to_string(const Plan& pl, char* buf, size_t n) {
                   pl.prec == fle::kPrecTF32 ? "tf32" : "3xtf32", pl.stages, pl.kps,
                   pl.tiles_a, pl.tiles_b, pl.num_kb, pl.dp_tiles, pl.sk_tiles, (long long)pl.sk_iters, pl.sk_grid,
                   pl.sk_slots, pl.grid, pl.ws_bytes);
+    if (pl.lo_mem) {
+        const size_t used = std::strlen(buf);
+        if (used + 1 < n) std::snprintf(buf + used, n - used, " xlo=mem");
+    }
     if (pl.mix_wide > 0) {
         const size_t used = std::strlen(buf);
         if (used + 1 < n)
@@ -681,6 +720,14 @@ size_t fle_workspace_size(int64_t M, int64_t K, int64_t N, const fle_epilogue_de
     DeviceInfo di;
     if (device_info(&di) != FLE_OK) return 0;
     return make_plan(M, K, N, d, di.sms, d->precision == FLE_PREC_3XTF32 ? di.pairs3x : di.pairs).ws_bytes;
+}
+
+size_t fle_workspace_size_min(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d) {
+    if (check_desc(d) != FLE_OK || check_shape(M, K, N, d) != FLE_OK) return 0;
+    if (M == 0 || N == 0 || K == 0) return 0;
+    DeviceInfo di;
+    if (device_info(&di) != FLE_OK) return 0;
+    return make_plan(M, K, N, d, di.sms, d->precision == FLE_PREC_3XTF32 ? di.pairs3x : di.pairs, false).ws_bytes;
 }
 
 int fle_plan_string(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, char* buf, size_t n) {
@@ -749,7 +796,11 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
         return cudaGetLastError() == cudaSuccess ? FLE_OK : FLE_ERR_CUDA;
     }
 
-    const Plan pl = make_plan(M, K, N, d, di.sms, d->precision == FLE_PREC_3XTF32 ? di.pairs3x : di.pairs);
+    const int pairs = d->precision == FLE_PREC_3XTF32 ? di.pairs3x : di.pairs;
+    Plan pl = make_plan(M, K, N, d, di.sms, pairs);
+    // a workspace too small for x's low parts (3xTF32) runs the plan that
+    // computes them inside the GEMM
+    if (pl.lo_mem && (!workspace || workspace_bytes < pl.ws_bytes)) pl = make_plan(M, K, N, d, di.sms, pairs, false);
     if (pl.ws_bytes > 0) {
         if (!workspace || workspace_bytes < pl.ws_bytes) return FLE_ERR_WORKSPACE;
         if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FLE_ERR_ALIGN;
@@ -765,6 +816,7 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
     p.sk_grid = pl.sk_grid;
     p.sk_slots = pl.sk_slots;
     p.tile_n = pl.bn;
+    p.lo_mem = pl.lo_mem ? 1 : 0;
     p.mix_wide = pl.mix_wide;
     std::memcpy(p.mix_a, pl.mix_a, sizeof p.mix_a);
     std::memcpy(p.mix_b, pl.mix_b, sizeof p.mix_b);
@@ -773,7 +825,7 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
         p.counters = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + pl.partial_bytes);
     }
 
-    CUtensorMap ta, tb, tb2, to;
+    CUtensorMap ta, tb, tb2, txlo, to;
     std::memset(&to, 0, sizeof to);
     // Elementwise kinds (direct or swapped layout) store through TMA when the
     // output rows are 16-byte multiples and the base is 16-byte aligned.
@@ -790,6 +842,14 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
     // tile (each CTA loads its 128 rows of both 256-wide sub-tiles)
     st = encode_operand(&tb, B, p.Nb, K, pl.pair ? (pl.bn > 256 ? 128 : pl.bn / 2) : pl.bn);
     if (st != FLE_OK) return st;
+    // x's low parts (3xTF32), in the workspace: the same boxes as x's own tiles
+    float* x_lo = pl.lo_mem ? reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.lo_offset) : nullptr;
+    txlo = ta;
+    if (pl.lo_mem) {
+        const int box = pl.swap ? (pl.pair ? (pl.bn > 256 ? 128 : pl.bn / 2) : pl.bn) : fle::kBM;
+        st = encode_operand(&txlo, x_lo, M, K, box);
+        if (st != FLE_OK) return st;
+    }
     // a mixed plan's 384-wide tiles: 64 rows per CTA of their 128-wide sub-tile
     tb2 = tb;
     if (pl.mix_wide > 0) {
@@ -804,6 +864,13 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
                      (long long)N, d->kind, line);
     }
 
+    if (pl.lo_mem) {
+        const int64_t n4 = M * K / 4;
+        const int64_t blocks = std::min<int64_t>((n4 + 255) / 256, 16 * static_cast<int64_t>(di.sms));
+        fle::fle_split_lo_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+            reinterpret_cast<const float4*>(x), reinterpret_cast<float4*>(x_lo), n4);
+        if (cudaGetLastError() != cudaSuccess) return FLE_ERR_CUDA;
+    }
     const bool prep = pool || pl.sk_tiles > 0;
     if (prep) {
         const int threads = 256;
@@ -813,7 +880,7 @@ int fle_forward(const float* x, const float* W, const float* b, int64_t M, int64
             pool ? out : nullptr, pool ? M : 0, p.counters, n_counters);
         if (cudaGetLastError() != cudaSuccess) return FLE_ERR_CUDA;
     }
-    if (dispatch(pl, ta, tb, tb2, to, p, prep, s) != cudaSuccess) return FLE_ERR_CUDA;
+    if (dispatch(pl, ta, tb, tb2, txlo, to, p, prep, s) != cudaSuccess) return FLE_ERR_CUDA;
     if (sync_check_enabled()) return fle_device_status(stream);
     return FLE_OK;
 }
@@ -1031,9 +1098,10 @@ extern "C" int fle_forward_noalloc(const float* x, const float* W, const float* 
         }
         scratch = g_noalloc_ptr[dev];
     }
-    // The plan's scratch need; 0 also for invalid arguments, which
-    // fle_forward then reports.
-    const size_t need = fle_workspace_size(M, K, N, d);
+    // The scratch need of the plan that fits the least workspace (3xTF32:
+    // x's low parts computed inside the GEMM); 0 also for invalid
+    // arguments, which fle_forward then reports.
+    const size_t need = fle_workspace_size_min(M, K, N, d);
     if (need > FLE_NOALLOC_SCRATCH_BYTES) return FLE_ERR_WORKSPACE;
     return fle_forward(x, W, b, M, K, N, d, out, scratch, FLE_NOALLOC_SCRATCH_BYTES, stream);
 }

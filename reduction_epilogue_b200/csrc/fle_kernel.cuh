@@ -85,6 +85,8 @@ struct KParams {
     int tma_out;            // direct layout: write out through TMA tile stores
     uint64_t timeout_ns;
     int tile_n;             // B rows per tile (the kernel's tile width)
+    int lo_mem;             // 3xTF32: the low parts of x are in memory (tensor map
+                            // tmXlo), copied with the tiles; the split warps split W only
     // Mixed-width plans of the 512-wide pair kernel (data-parallel only):
     // each 256-row panel r holds mix_a[r] tiles 512 wide from column 0, then
     // mix_b[r] tiles 384 wide.  Units [0, mix_wide) are the 512-wide tiles,
@@ -210,6 +212,7 @@ struct Cfg {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128 is a multiple of 16 in [16,256]");
     static_assert(kABytes % 1024 == 0 && kBBytes % 1024 == 0, "tiles must keep 1024-byte alignment");
     static_assert(kSmemBytes <= 232448, "exceeds 227 KB of shared memory per block");
+    static_assert(PREC != kPrec3xTF32 || KPS == 1, "3xTF32 stages hold one k-block");
 };
 
 // ----------------------------------------------------------------------------
@@ -557,6 +560,22 @@ __device__ __forceinline__ void split_lo_parts(const float4* __restrict__ x4, fl
     }
 }
 
+// The low parts of x for 3xTF32, written once per call into the workspace
+// and copied with the tiles (each x tile is otherwise split again by every
+// CTA that multiplies it): lo = x - (x with the low 13 mantissa bits
+// cleared), the same value split_lo_parts computes.  n4: float4 of x.
+__global__ void __launch_bounds__(256) fle_split_lo_kernel(const float4* __restrict__ x, float4* __restrict__ lo,
+                                                           int64_t n4) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float4 v = x[i];
+        lo[i] = make_float4(v.x - __uint_as_float(__float_as_uint(v.x) & 0xFFFFE000u),
+                            v.y - __uint_as_float(__float_as_uint(v.y) & 0xFFFFE000u),
+                            v.z - __uint_as_float(__float_as_uint(v.z) & 0xFFFFE000u),
+                            v.w - __uint_as_float(__float_as_uint(v.w) & 0xFFFFE000u));
+    }
+}
+
 // Barrier among the eight epilogue warps only (named barrier 1, 256 threads).
 __device__ __forceinline__ void epilogue_bar_sync() {
     asm volatile("bar.sync 1, 256;" ::: "memory");
@@ -590,7 +609,8 @@ __device__ __forceinline__ bool sk_take_own(const KParams& p, const unsigned* co
 template <int BN, int PREC, bool SWAP, int KPS>
 __global__ void __launch_bounds__(kThreads, 1)
 fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmOut, const KParams p) {
+                const __grid_constant__ CUtensorMap tmXlo, const __grid_constant__ CUtensorMap tmOut,
+                const KParams p) {
     using C = Cfg<BN, PREC, SWAP, KPS>;
     constexpr int S = C::kStages;
     constexpr uint32_t kIdesc = idesc_tf32(kBM, BN);
@@ -643,6 +663,7 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         fence_barrier_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if (PREC == kPrec3xTF32 && p.lo_mem) tma_prefetch_desc(&tmXlo);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
@@ -676,10 +697,23 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         if (mbar_test_wait(bar_full(stage), phase)) record_error(kErrProtocol, kWhereProdEmpty);
                         stage_tag[stage] = work_tag(u.t, kb);
                     }
-                    mbar_arrive_expect_tx(bar_full(stage), n * C::kKbBytes);
+                    // 3xTF32 with x's low parts in memory: they are copied into
+                    // the low half beside the tiles (x is B in the swapped
+                    // order, A in the direct one)
+                    const uint32_t xlo_bytes =
+                        (PREC == kPrec3xTF32 && p.lo_mem) ? static_cast<uint32_t>(SWAP ? C::kBBytes : C::kABytes) : 0u;
+                    mbar_arrive_expect_tx(bar_full(stage), n * (C::kKbBytes + xlo_bytes));
                     for (int j = 0; j < n; ++j) {
                         tma_load_2d(sA(stage) + j * C::kABytes, &tmA, bar_full(stage), (kb + j) * kBK, u.ta * kBM);
                         tma_load_2d(sB(stage) + j * C::kBBytes, &tmB, bar_full(stage), (kb + j) * kBK, u.tb * BN);
+                        if (xlo_bytes) {
+                            if constexpr (SWAP)
+                                tma_load_2d(sB(stage) + C::kLoadBytes + j * C::kBBytes, &tmXlo, bar_full(stage),
+                                            (kb + j) * kBK, u.tb * BN);
+                            else
+                                tma_load_2d(sA(stage) + C::kLoadBytes + j * C::kABytes, &tmXlo, bar_full(stage),
+                                            (kb + j) * kBK, u.ta * kBM);
+                        }
                     }
                     ++fills;
                     if (++stage == S) { stage = 0; phase ^= 1u; }
@@ -803,7 +837,13 @@ fle_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     // operand-conversion test).
                     const float4* x4 = reinterpret_cast<const float4*>(smem + stage * C::kStageBytes);
                     float4* lo4 = reinterpret_cast<float4*>(smem + stage * C::kStageBytes + C::kLoadBytes);
-                    split_lo_parts<C::kLoadBytes / 16>(x4, lo4, ct);
+                    if (p.lo_mem) {
+                        // only W's tile: A in the swapped order, B in the direct one
+                        constexpr int kWOff = SWAP ? 0 : C::kABytes / 16;
+                        split_lo_parts<(SWAP ? C::kABytes : C::kBBytes) / 16>(x4 + kWOff, lo4 + kWOff, ct);
+                    } else {
+                        split_lo_parts<C::kLoadBytes / 16>(x4, lo4, ct);
+                    }
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar_conv(stage));

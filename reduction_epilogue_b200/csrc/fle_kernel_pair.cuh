@@ -90,8 +90,8 @@ struct PairCfg {
 template <int PREC, int KPS, int BN, bool SWAP>
 __global__ void __launch_bounds__(kThreads, 1)
 fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmOut,
-                     const KParams p) {
+                     const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmXlo,
+                     const __grid_constant__ CUtensorMap tmOut, const KParams p) {
     using C = PairCfg<PREC, KPS, BN, SWAP>;
     constexpr bool k3x = (PREC == kPrec3xTF32);
     constexpr int S = C::kStages;
@@ -160,6 +160,7 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
         if (kWide && p.mix_wide > 0) tma_prefetch_desc(&tmB2);
+        if (k3x && p.lo_mem) tma_prefetch_desc(&tmXlo);
     }
     if (warp == 1) {
         tmem_alloc_pair(smem_u32(tmem_slot), C::kTmemCols);
@@ -205,14 +206,25 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                         fence_acq_rel_cluster();
                     }
                     if constexpr (k3x) {
-                        // own barrier: this CTA's split warps wait for these bytes
-                        mbar_arrive_expect_tx(bar_full(stage), n * C::kKbBytes);
+                        // own barrier: this CTA's split warps wait for these bytes;
+                        // x's low parts, when in memory, come with them into the
+                        // low half (x is B in the swapped order, A in the direct one)
+                        const uint32_t xlo_bytes = p.lo_mem ? static_cast<uint32_t>(SWAP ? C::kBBytes : C::kABytes) : 0u;
+                        mbar_arrive_expect_tx(bar_full(stage), n * (C::kKbBytes + xlo_bytes));
                         for (int j = 0; j < n; ++j) {
                             tma_load_2d(sA(stage) + j * C::kABytes, &tmA, bar_full(stage), (kb + j) * kBKW, ra);
 #pragma unroll
                             for (int sb = 0; sb < C::kNSub; ++sb)
                                 tma_load_2d(sB(stage) + j * C::kBBytes + sb * C::kSubBBytes, &tmB, bar_full(stage),
                                             (kb + j) * kBKW, rb + sb * C::kSubN);
+                            if (xlo_bytes) {
+                                if constexpr (SWAP)
+                                    tma_load_2d(sB(stage) + C::kLoadBytes + j * C::kBBytes, &tmXlo, bar_full(stage),
+                                                (kb + j) * kBKW, rb);
+                                else
+                                    tma_load_2d(sA(stage) + C::kLoadBytes + j * C::kABytes, &tmXlo, bar_full(stage),
+                                                (kb + j) * kBKW, ra);
+                            }
                         }
                     } else {
                         // the leader expects both CTAs' bytes on its own full barrier
@@ -363,7 +375,13 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     }
                     const float4* x4 = reinterpret_cast<const float4*>(smem + stage * C::kStageBytes);
                     float4* lo4 = reinterpret_cast<float4*>(smem + stage * C::kStageBytes + C::kLoadBytes);
-                    split_lo_parts<C::kLoadBytes / 16>(x4, lo4, ct);
+                    if (p.lo_mem) {
+                        // only W's tile: A in the swapped order, B in the direct one
+                        constexpr int kWOff = SWAP ? 0 : C::kABytes / 16;
+                        split_lo_parts<(SWAP ? C::kABytes : C::kBBytes) / 16>(x4 + kWOff, lo4 + kWOff, ct);
+                    } else {
+                        split_lo_parts<C::kLoadBytes / 16>(x4, lo4, ct);
+                    }
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) mbar_arrive_cluster(mapa_shared(bar_split(stage), 0));
