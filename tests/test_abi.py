@@ -144,6 +144,10 @@ def test_empty_sizes_enqueue_nothing(lib):
     assert _call(lib, 4, 8, 0, d, x=None, W=None, out=None) == 0
     assert lib.fle_workspace_size(0, 8, 8, ctypes.byref(d)) == 0
     assert lib.fle_workspace_size(4, 6, 8, ctypes.byref(d)) == 0
+    lib.fle_workspace_size_min.restype = ctypes.c_size_t
+    assert lib.fle_workspace_size_min(0, 8, 8, ctypes.byref(d)) == 0
+    assert lib.fle_workspace_size_min(4, 6, 8, ctypes.byref(d)) == 0
+    assert lib.fle_workspace_size_min(-1, 8, 8, ctypes.byref(d)) == 0  # invalid: 0, fle_forward reports it
 
 
 def test_binding_raises_with_status():
