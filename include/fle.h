@@ -186,8 +186,8 @@ int fle_forward_pooled(const float* x, const float* W, const float* b,
 /* Bytes of caller workspace for the fastest plan of these arguments (0 when
  * the plan needs none): split-K partial tiles and arrival counters, and in
  * 3xTF32 the low parts of x (M x K fp32, written by a pre-pass so that the
- * GEMM splits only W).  Returns 0 for invalid arguments too; fle_forward then
- * reports the argument error. */
+ * GEMM splits only W; not for M <= 64 or x above 1 GiB).  Returns 0 for
+ * invalid arguments too; fle_forward then reports the argument error. */
 size_t fle_workspace_size(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* desc);
 
 /* The least workspace fle_forward accepts for these arguments: the plan

@@ -498,15 +498,18 @@ Plan make_plan_core(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d,
 
 // 3xTF32: x's low parts are split once per call into the workspace, except
 // for skinny swapped shapes (M <= 64), where x is a small part of each stage
-// and the pre-pass does not pay (measured no faster at M = 16).  Measured
+// and the pre-pass does not pay (measured no faster at M = 16), and for x
+// above 1 GiB, whose low parts would make the workspace as large.  Measured
 // with the low parts in memory: 2048 x 8192 x 8192 1358 -> ~1066 us of GEMM,
 // 128 x 32768 x 32768 1766 -> ~1565 us, M = 256 239 -> ~198 us.
 Plan make_plan(int64_t M, int64_t K, int64_t N, const fle_epilogue_desc* d, int sms, int pairs, bool lo_mem) {
     Plan pl = make_plan_core(M, K, N, d, sms, pairs);
-    if (lo_mem && pl.prec == fle::kPrec3xTF32 && K > 0 && !(pl.swap && M <= 64) && !lo_mem_disabled()) {
+    const size_t x_bytes = static_cast<size_t>(M) * static_cast<size_t>(K) * sizeof(float);
+    if (lo_mem && pl.prec == fle::kPrec3xTF32 && K > 0 && !(pl.swap && M <= 64) && x_bytes <= (size_t(1) << 30) &&
+        !lo_mem_disabled()) {
         pl.lo_mem = true;
         pl.lo_offset = (pl.ws_bytes + 255) & ~size_t(255);
-        pl.ws_bytes = pl.lo_offset + static_cast<size_t>(M) * static_cast<size_t>(K) * sizeof(float);
+        pl.ws_bytes = pl.lo_offset + x_bytes;
     }
     return pl;
 }
