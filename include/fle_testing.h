@@ -51,10 +51,11 @@ int fle_test_epilogue_math(const float* in, float* out, int64_t n, int32_t which
  *   FLE_FINISH_LAST: by whichever contributor arrives last, which sums all
  *                    parked partials starting from zero.
  * Both give the same result (partials are summed in contributor order).
- * With FLE_FINISH_AUTO (the default) timing decides per tile and no CTA
- * waits for another.  FLE_FINISH_OWN makes the k-block-0 CTA wait, up to a
- * fixed 50 ms, for the others before deciding (it parks if they have not
- * arrived by then); FLE_FINISH_LAST makes it always park.
+ * With FLE_FINISH_AUTO (the default) the k-block-0 CTA waits up to 20 us for
+ * the others to arrive, then decides; timing decides per tile.
+ * FLE_FINISH_OWN makes that wait up to 50 ms, so that it finishes whenever
+ * the others arrive (it parks if they have not by then); FLE_FINISH_LAST makes
+ * it always park.
  * fle_test_set_finisher sets the mode for later fle_forward calls in this
  * process (all devices) and returns the previous one, or -1 for an unknown
  * mode (nothing changes).
