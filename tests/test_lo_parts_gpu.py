@@ -8,8 +8,8 @@ W's tiles; with fle_workspace_size_min() bytes the split warps compute both,
 as every CTA's tiles arrive.  The tensor core then reads identical operands,
 so the two must agree bit for bit, and both must meet the 3xTF32 bound
 against the oracle.  Covered: direct tiles on CTA pairs (whole, split along
-K, ragged), the row-max kind, the swapped one-CTA kernel, and a skinny shape
-(M <= 64) whose plan keeps the split inside the GEMM.
+K, ragged, large M), the row-max kind, the swapped one-CTA kernel, and a
+skinny shape (M <= 64) whose plan keeps the split inside the GEMM.
 """
 import numpy as np
 import pytest
@@ -27,6 +27,8 @@ SHAPES = [
     (100, 1056, 520, "swish_scale", True),                 # swapped one-CTA tiles
     (128, 8192, 4096, "scale_hardtanh_gelu", True),        # swapped, tiles split along K
     (48, 4096, 3000, "none", False),                       # M <= 64: split inside the GEMM
+    (2048, 1024, 2048, "scale_hardtanh_gelu", True),       # large M on pairs
+    (2100, 1028, 1500, "swish_scale", True),               # the same, ragged M, K and N
 ]
 
 
@@ -51,17 +53,18 @@ def test_low_parts_in_memory_match_the_split_in_the_gemm(fle, M, K, N, problem, 
         assert full >= least + 4 * M * K, (full, least)
     else:
         assert full == least
+    sizes = [full, least]
     x, W, b = synth.linear_inputs(M, K, N, seed=M + K + N + 3, device="cuda")
     shape = (M,) if problem.startswith("avgpool") else (M, N)
     outs = []
-    for ws_bytes in (full, least):
+    for ws_bytes in sizes:
         ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device="cuda")
         out = torch.full(shape, float("nan"), device="cuda")
         fle.forward(x, W, b, out, d, workspace=ws, workspace_bytes=ws_bytes)
         torch.cuda.synchronize()
         assert fle.device_status() == 0, (ws_bytes, plan)
         outs.append(out)
-    assert torch.equal(outs[0], outs[1]), plan
+    assert all(torch.equal(outs[0], o) for o in outs[1:]), plan
     rows = synth.sample_rows(M, M if problem.startswith("avgpool") else 24, seed=8)
     ref = oracle.forward_rows(x.cpu().numpy(), W.cpu().numpy(), b.cpu().numpy(), rows=rows, **oracle.PROBLEMS[problem])
     got = outs[0].cpu().numpy()[rows].astype(np.float64)
