@@ -260,7 +260,9 @@ bool mixed_cut(int64_t panels, int64_t N, int64_t G, unsigned char* a_out, unsig
                int* n_narrow) {
     if (panels < 1 || panels > fle::kMaxMixPanels || G < 1) return false;
     const int64_t A = (N + fle::kMixWide - 1) / fle::kMixWide;
-    if (A > 255) return false;
+    // at most one tile of each width per pair: no cut exists beyond 2G tiles
+    // of 512 (this also bounds the search below: A <= 2G / panels)
+    if (A > 255 || panels * A > 2 * G) return false;
     auto b_of = [&](int64_t a) {
         const int64_t rest = N - fle::kMixWide * a;
         return rest > 0 ? (rest + fle::kMixNarrow - 1) / fle::kMixNarrow : int64_t(0);
@@ -268,7 +270,7 @@ bool mixed_cut(int64_t panels, int64_t N, int64_t G, unsigned char* a_out, unsig
     int64_t best_wide = -1, best_spread = 0, best_a1 = 0, best_a2 = 0, best_n1 = 0;
     for (int64_t a1 = 0; a1 <= A; ++a1)
         for (int64_t a2 = a1; a2 <= A; ++a2)
-            for (int64_t n1 = (a1 == a2 ? panels : 1); n1 <= panels; ++n1) {
+            for (int64_t n1 = (a1 == a2 ? panels : 1); n1 <= (a1 == a2 ? panels : panels - 1); ++n1) {
                 const int64_t wide = n1 * a1 + (panels - n1) * a2;
                 const int64_t narrow = n1 * b_of(a1) + (panels - n1) * b_of(a2);
                 if (wide > G || narrow > G || b_of(a1) > 255) continue;
