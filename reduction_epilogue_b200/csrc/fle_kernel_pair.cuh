@@ -384,7 +384,14 @@ fle_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     }
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(mapa_shared(bar_split(stage), 0));
+                    // the leader's split warps arrive on their own CTA's barrier
+                    // at CTA scope; only the peer's need a cluster-scope release
+                    if (lane == 0) {
+                        if (rank == 0)
+                            mbar_arrive(bar_split(stage));
+                        else
+                            mbar_arrive_cluster(mapa_shared(bar_split(stage), 0));
+                    }
                     if (++stage == S) { stage = 0; phase ^= 1u; }
                 }
             }
